@@ -1,0 +1,357 @@
+"""Benchmark: Sliding Tile Attention forward on B200.
+
+Metric: STA forward ms per call and useful TFLOP/s on the 30x48x80 video latent
+(24 heads, d=128, tile 6x8x8, window 3x3x3), with useful FLOPs
+4 * N * keys_per_query * d per head, and the fraction of the measured dense
+BF16 tensor-core peak.  One step = one sta_forward call (the whole hot path:
+K/V gather, QK^T, softmax, PV, O/LSE write-back) on inputs resident in HBM.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        python bench.py --impl reference ...   (the fp64 CPU oracle arm)
+Multi-GPU: launched by torchrun, one rank per GPU; every rank runs its own
+independent problem (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sparse_local_attention_b200.workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "STA fwd ms and useful TFLOPS at 30×48×80, 24 heads, d=128; % of BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sta_fwd_kernel_dit720p.md")
+KERNEL_SOURCE = os.path.join(ROOT, "sparse_local_attention_b200", "csrc", "sta_fwd.cu")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the forward kernel from the committed ncu
+    summary, if it was taken on this workload with the current kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    txt = open(PROFILE_SUMMARY).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s+workload:\s*(\S+)\s+kernel_sha:\s*(\w+)", txt)
+    if not m or m.group(2) != workload or m.group(3) != kernel_hash():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, local):
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return dist
+    return None
+
+
+def max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_sample_rows(wl, n_rows: int):
+    """First n_rows query rows of the first (batch, head) slice, tile by tile
+    from the middle of the grid (interior windows)."""
+    from sparse_local_attention_b200.workloads import tile_tokens
+    rows, tile = [], wl.n_tiles // 2
+    while len(rows) < n_rows:
+        rows.extend(tile_tokens(wl, tile % wl.n_tiles))
+        tile += 1
+    return np.array(rows[:n_rows], dtype=np.int64)
+
+
+def time_oracle(wl, q, k, v, target_s: float):
+    """Time the oracle (as it stands) on a bounded sample of the workload and
+    return (TFLOP/s, sample description, threads)."""
+    import oracle
+    g = oracle.Geometry(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows))
+    flops_per_row = 4.0 * wl.keys_per_query(0) * wl.d
+    n = 64
+    t0 = time.perf_counter()
+    oracle.forward(g, q, k, v, rows=oracle_sample_rows(wl, n))
+    dt = time.perf_counter() - t0
+    n2 = int(max(n, min(wl.N, n * target_s / max(dt, 1e-3))))
+    rows = oracle_sample_rows(wl, n2)
+    t0 = time.perf_counter()
+    oracle.forward(g, q, k, v, rows=rows)
+    dt = time.perf_counter() - t0
+    tflops = flops_per_row * len(rows) / dt / 1e12
+    return tflops, dt, f"{len(rows)} query rows of head 0 ({wl.keys_per_query(0)} keys each), {dt:.1f} s", oracle.threads()
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    import oracle
+    q, k, v = make_inputs(wl)
+    g = oracle.Geometry(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows))
+    rows = oracle_sample_rows(wl, args.ref_rows)
+    flops = 4.0 * wl.keys_per_query(0) * wl.d * len(rows)
+    for _ in range(args.warmup):
+        oracle.forward(g, q, k, v, rows=rows)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(g, q, k, v, rows=rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    sample = f"{len(rows)} query rows of head 0 per step ({wl.keys_per_query(0)} keys each)"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: {wl.description}", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    from sparse_local_attention_b200 import sta
+
+    world, rank, local = dist_env()
+    dist = init_dist(world, local)
+    torch.cuda.set_device(local)
+    wl = WORKLOADS[args.workload]
+    pk, pk_kind = peaks()
+
+    q_h, k_h, v_h = (x.pin_memory() for x in make_inputs(wl, seed=rank))
+    q, k, v = (x.cuda() for x in (q_h, k_h, v_h))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False))
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32, device="cuda")
+    ws = plan.workspace()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sta.sta_forward(plan, q, k, v, o, lse, ws, stream)
+
+    sta.sta_forward(plan, q, k, v, o, lse, ws, stream, check=True)  # one checked call
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms_rank = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(dist, ms_rank)
+    flops = wl.forward_flops()
+    value = flops * world / (ms * 1e-3) / 1e12
+    launches_per_step = 1
+
+    # --- end to end through the public API: pinned host in, host out
+    o_h = torch.empty_like(q_h).pin_memory()
+    lse_h = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32).pin_memory()
+    q2, k2, v2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        q2.copy_(q_h, non_blocking=True)
+        k2.copy_(k_h, non_blocking=True)
+        v2.copy_(v_h, non_blocking=True)
+        sta.sta_forward(plan, q2, k2, v2, o, lse, ws, stream)
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / e2e_steps)
+    h2d = 3 * q.numel() * 2
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    # --- dense full-attention baseline on the same shapes (library SDPA)
+    dense = None
+    if not args.no_dense and rank == 0:
+        torch.backends.cuda.enable_flash_sdp(True)
+        for _ in range(2):
+            torch.nn.functional.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        d0.record(stream)
+        for _ in range(reps):
+            torch.nn.functional.scaled_dot_product_attention(q, k, v)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = d0.elapsed_time(d1) / reps
+        dflops = 4.0 * wl.N * wl.N * wl.d * wl.Hh * wl.B
+        dense = {"impl": "torch.nn.functional.scaled_dot_product_attention (full 3D attention, bf16)",
+                 "ms": dms, "tflops": dflops / (dms * 1e-3) / 1e12, "speedup_sta_vs_dense": dms / ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tflops, dt, sample, cores = time_oracle(wl, q_h, k_h, v_h, args.cpu_seconds)
+        cpu = {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    clocks = clk.summary()
+    if rank == 0:
+        peak_key = "bf16_tflops"
+        peak = float(pk.get(peak_key, FALLBACK_PEAKS[peak_key]))
+        achieved = flops / (ms * 1e-3) / 1e12
+        traffic = profiled_traffic(wl.name)
+        out = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {wl.description}", "useful_tflop_per_step_per_gpu": flops / 1e12,
+                       "l2": "inputs 3 x %.0f MB per GPU, larger than the 126 MB L2; no flush" % (q.numel() * 2 / 1e6),
+                       "parallelism": f"independent problem per GPU x{world}"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{pk_kind} {peak_key}", "kernel": "sta_fwd_kernel"},
+            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "dense_baseline": dense,
+        }
+        print(json.dumps(out), flush=True)
+    plan.destroy()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=384)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,469 @@
+// sta_api.cpp -- host side of libsta.so: argument checking, the planner
+// (window starts, KV-tile lists, inverse lists, work order), TMA descriptors
+// and kernel launches behind the C ABI of include/sta.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <numeric>
+#include <vector>
+
+#include "../../include/sta.h"
+#include "sta_kernels.h"
+
+using sta::Geometry;
+
+struct sta_plan_s {
+  sta_problem p{};
+  Geometry g{};
+  std::vector<int32_t> window;   // heads*3, as given
+  std::vector<int32_t> wclamp;   // heads*3, clamped to the grid
+  std::vector<int32_t> count;    // heads: key tiles per query tile
+  int32_t kv_stride = 0;         // max(count)
+  std::vector<int32_t> kv_list;  // [heads][n_tiles][kv_stride]
+  std::vector<int32_t> inv_off;  // [heads][n_tiles + 1], absolute into inv_idx
+  std::vector<int32_t> inv_idx;
+  std::vector<int2> work;        // forward work items
+  int nqb = 1;
+  int kv_mode = sta::kKvTiled2D;
+  int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
+  bool host_only = false;
+  bool tiled = false;
+  float scale = 0.f;
+  int device = -1, num_sms = 0;
+  // device copies
+  int32_t *d_kv_list = nullptr, *d_count = nullptr, *d_inv_off = nullptr, *d_inv_idx = nullptr;
+  int2 *d_work = nullptr;
+};
+
+namespace {
+
+uint64_t g_wait_limit_ns = 2000ull * 1000 * 1000;  // 2 s per barrier wait
+
+// Start of the window of `w` tiles (already clamped to G) around tile q,
+// shifted inward so that [start, start + w) stays inside [0, G).
+inline int window_start(int q, int w, int G) {
+  int s = q - w / 2;
+  if (s < 0) s = 0;
+  if (s > G - w) s = G - w;
+  return s;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t tensor_bytes(const sta_plan_s *pl) {
+  return (size_t)pl->g.B * pl->g.Hh * pl->g.N * pl->g.d * 2;
+}
+
+constexpr size_t kStatusBytes = 256;
+
+size_t fwd_workspace(const sta_plan_s *pl) {
+  size_t b = kStatusBytes;
+  if (!pl->tiled && pl->kv_mode == sta::kKvTiled2D) b += 2 * tensor_bytes(pl);
+  return b;
+}
+
+size_t bwd_workspace(const sta_plan_s *pl) {
+  return kStatusBytes;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D map over a tile-major [rows][d] bf16 buffer, box 64 x piece_rows, 128B swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const Geometry &g = pl->g;
+  cuuint64_t dims[2] = {(cuuint64_t)g.d, (cuuint64_t)g.B * g.Hh * g.N};
+  cuuint64_t strides[1] = {(cuuint64_t)g.d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)pl->piece_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 5D map (d, W, H, T, B*Hh) over a raster tensor; one box = one piece of a tile.
+bool make_map_5d(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const Geometry &g = pl->g;
+  const cuuint64_t row = (cuuint64_t)g.d * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T,
+                        (cuuint64_t)g.B * g.Hh};
+  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * (cuuint64_t)g.N};
+  cuuint32_t box[5] = {64, (cuuint32_t)pl->box_w, (cuuint32_t)pl->box_h, (cuuint32_t)pl->box_t, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+void free_device(sta_plan_s *pl) {
+  cudaFree(pl->d_kv_list);
+  cudaFree(pl->d_count);
+  cudaFree(pl->d_inv_off);
+  cudaFree(pl->d_inv_idx);
+  cudaFree(pl->d_work);
+  pl->d_kv_list = pl->d_count = pl->d_inv_off = pl->d_inv_idx = nullptr;
+  pl->d_work = nullptr;
+}
+
+template <class T>
+bool upload(T **dst, const std::vector<T> &src) {
+  if (src.empty()) return true;
+  if (cudaMalloc(reinterpret_cast<void **>(dst), src.size() * sizeof(T)) != cudaSuccess) return false;
+  return cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice) == cudaSuccess;
+}
+
+int gcd_int(int a, int b) {
+  while (b) {
+    int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
+// Plan the TMA gather of one piece of `rows` tokens of a tile directly from
+// the raster tensor: the piece must be a box (whole w-runs, whole h-planes).
+bool raster_box(const Geometry &g, int rows, int *bw, int *bh, int *bt) {
+  const int plane = g.th * g.tw;
+  if (rows % plane == 0) {
+    const int t = rows / plane;
+    if (g.tt % t) return false;
+    *bw = g.tw, *bh = g.th, *bt = t;
+  } else if (rows % g.tw == 0 && rows < plane) {
+    const int h = rows / g.tw;
+    if (g.th % h) return false;
+    *bw = g.tw, *bh = h, *bt = 1;
+  } else if (rows < g.tw && g.tw % rows == 0) {
+    *bw = rows, *bh = 1, *bt = 1;
+  } else {
+    return false;
+  }
+  return *bw <= 256 && *bh <= 256 && *bt <= 256;
+}
+
+sta_status finish_call(const sta_plan_s *pl, void *workspace, cudaStream_t stream, uint32_t flags) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return STA_ERR_CUDA;
+  if (flags & STA_CALL_CHECK) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return STA_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpy(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return STA_ERR_CUDA;
+    if (st != 0) return STA_ERR_TIMEOUT;
+  }
+  (void)pl;
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sta_status_string(sta_status s) {
+  switch (s) {
+    case STA_OK: return "ok";
+    case STA_ERR_INVALID_ARG: return "invalid argument";
+    case STA_ERR_SHAPE: return "shape not supported (tile must divide the latent; sizes must be >= 1)";
+    case STA_ERR_UNSUPPORTED: return "unsupported configuration (head_dim must be 64 or 128; tile volume a multiple of 8; sm_100 device)";
+    case STA_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case STA_ERR_WORKSPACE: return "workspace missing or too small";
+    case STA_ERR_OOM: return "out of memory";
+    case STA_ERR_CUDA: return "CUDA runtime error";
+    case STA_ERR_TIMEOUT: return "kernel wait timed out; outputs are invalid";
+  }
+  return "unknown status";
+}
+
+void sta_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
+  if (!prob || !out || !prob->window) return STA_ERR_INVALID_ARG;
+  const uint32_t known = STA_PROBLEM_BACKWARD | STA_PROBLEM_TILED | STA_PROBLEM_HOST_ONLY;
+  if (prob->flags & ~known) return STA_ERR_INVALID_ARG;
+  if (prob->batch < 1 || prob->heads < 1 || prob->T < 1 || prob->H < 1 || prob->W < 1 || prob->tile_t < 1 ||
+      prob->tile_h < 1 || prob->tile_w < 1)
+    return STA_ERR_SHAPE;
+  if (prob->T % prob->tile_t || prob->H % prob->tile_h || prob->W % prob->tile_w) return STA_ERR_SHAPE;
+  if (prob->head_dim != 64 && prob->head_dim != 128) return STA_ERR_UNSUPPORTED;
+  for (int i = 0; i < 3 * prob->heads; ++i)
+    if (prob->window[i] < 1) return STA_ERR_INVALID_ARG;
+  const long long N = (long long)prob->T * prob->H * prob->W;
+  const long long rows = N * prob->batch * prob->heads;
+  if (rows >= (1ll << 31) - 1024) return STA_ERR_SHAPE;
+  const long long tau = (long long)prob->tile_t * prob->tile_h * prob->tile_w;
+  if (tau % 8) return STA_ERR_UNSUPPORTED;
+
+  sta_plan_s *pl = new (std::nothrow) sta_plan_s();
+  if (!pl) return STA_ERR_OOM;
+  pl->p = *prob;
+  pl->host_only = (prob->flags & STA_PROBLEM_HOST_ONLY) != 0;
+  pl->tiled = (prob->flags & STA_PROBLEM_TILED) != 0;
+  Geometry &g = pl->g;
+  g.B = prob->batch, g.Hh = prob->heads, g.d = prob->head_dim, g.N = (int)N;
+  g.T = prob->T, g.H = prob->H, g.W = prob->W;
+  g.tt = prob->tile_t, g.th = prob->tile_h, g.tw = prob->tile_w;
+  g.GT = g.T / g.tt, g.GH = g.H / g.th, g.GW = g.W / g.tw;
+  g.n_tiles = g.GT * g.GH * g.GW;
+  g.tau = (int)tau;
+  pl->scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt((float)g.d);
+  pl->nqb = (g.tau + 127) / 128;
+
+  try {
+    // --- per-head clamped windows and list lengths
+    pl->window.assign(prob->window, prob->window + 3 * g.Hh);
+    pl->wclamp.resize(3 * g.Hh);
+    pl->count.resize(g.Hh);
+    const int G[3] = {g.GT, g.GH, g.GW};
+    for (int h = 0; h < g.Hh; ++h) {
+      int c = 1;
+      for (int a = 0; a < 3; ++a) {
+        pl->wclamp[3 * h + a] = std::min(pl->window[3 * h + a], G[a]);
+        c *= pl->wclamp[3 * h + a];
+      }
+      pl->count[h] = c;
+    }
+    pl->kv_stride = *std::max_element(pl->count.begin(), pl->count.end());
+
+    // --- forward KV-tile lists: whole key tiles of each query tile's window,
+    //     ascending tile-major index (t outer, w inner)
+    pl->kv_list.assign((size_t)g.Hh * g.n_tiles * pl->kv_stride, -1);
+    for (int h = 0; h < g.Hh; ++h) {
+      const int *w = &pl->wclamp[3 * h];
+      for (int qt = 0; qt < g.GT; ++qt)
+        for (int qh = 0; qh < g.GH; ++qh)
+          for (int qw = 0; qw < g.GW; ++qw) {
+            const int qtile = (qt * g.GH + qh) * g.GW + qw;
+            const int st = window_start(qt, w[0], g.GT), sh = window_start(qh, w[1], g.GH),
+                      sw = window_start(qw, w[2], g.GW);
+            int32_t *dst = &pl->kv_list[((size_t)h * g.n_tiles + qtile) * pl->kv_stride];
+            int n = 0;
+            for (int kt = st; kt < st + w[0]; ++kt)
+              for (int kh = sh; kh < sh + w[1]; ++kh)
+                for (int kw = sw; kw < sw + w[2]; ++kw) dst[n++] = (kt * g.GH + kh) * g.GW + kw;
+          }
+    }
+
+    // --- inverse lists (key tile -> query tiles), CSR per head
+    if (prob->flags & STA_PROBLEM_BACKWARD) {
+      pl->inv_off.assign((size_t)g.Hh * (g.n_tiles + 1), 0);
+      std::vector<std::vector<int32_t>> buckets(g.n_tiles);
+      for (int h = 0; h < g.Hh; ++h) {
+        for (auto &b : buckets) b.clear();
+        for (int qtile = 0; qtile < g.n_tiles; ++qtile) {
+          const int32_t *lst = &pl->kv_list[((size_t)h * g.n_tiles + qtile) * pl->kv_stride];
+          for (int i = 0; i < pl->count[h]; ++i) buckets[lst[i]].push_back(qtile);
+        }
+        int32_t *off = &pl->inv_off[(size_t)h * (g.n_tiles + 1)];
+        off[0] = (int32_t)pl->inv_idx.size();
+        for (int k = 0; k < g.n_tiles; ++k) {
+          pl->inv_idx.insert(pl->inv_idx.end(), buckets[k].begin(), buckets[k].end());
+          off[k + 1] = (int32_t)pl->inv_idx.size();
+        }
+      }
+    }
+
+    // --- forward work items, heaviest heads first (longest-processing-time
+    //     order for the persistent grid); within a head, (batch, tile, block)
+    std::vector<int> heads(g.Hh);
+    std::iota(heads.begin(), heads.end(), 0);
+    std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
+    pl->work.reserve((size_t)g.B * g.Hh * g.n_tiles * pl->nqb);
+    for (int h : heads)
+      for (int b = 0; b < g.B; ++b)
+        for (int t = 0; t < g.n_tiles; ++t)
+          for (int qb = 0; qb < pl->nqb; ++qb) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->nqb + qb));
+  } catch (const std::bad_alloc &) {
+    delete pl;
+    return STA_ERR_OOM;
+  }
+
+  // --- how K/V tiles reach shared memory
+  pl->piece_rows = gcd_int(g.tau, 128);
+  if (pl->tiled) {
+    pl->kv_mode = sta::kKvTiled2D;
+  } else if (raster_box(g, pl->piece_rows, &pl->box_w, &pl->box_h, &pl->box_t)) {
+    pl->kv_mode = sta::kKvRaster5D;
+  } else {
+    pl->kv_mode = sta::kKvTiled2D;  // permute K and V into the workspace first
+  }
+
+  if (!pl->host_only) {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&pl->num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      delete pl;
+      return STA_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) {
+      delete pl;
+      return STA_ERR_UNSUPPORTED;
+    }
+    pl->device = dev;
+    std::vector<int32_t> cnt(pl->count);
+    if (!upload(&pl->d_kv_list, pl->kv_list) || !upload(&pl->d_count, cnt) || !upload(&pl->d_work, pl->work) ||
+        !upload(&pl->d_inv_off, pl->inv_off) || !upload(&pl->d_inv_idx, pl->inv_idx)) {
+      cudaError_t e = cudaGetLastError();
+      free_device(pl);
+      delete pl;
+      return e == cudaErrorMemoryAllocation ? STA_ERR_OOM : STA_ERR_CUDA;
+    }
+  }
+  *out = pl;
+  return STA_OK;
+}
+
+sta_status sta_plan_destroy(sta_plan_t pl) {
+  if (!pl) return STA_OK;
+  if (!pl->host_only) free_device(pl);
+  delete pl;
+  return STA_OK;
+}
+
+sta_status sta_plan_workspace_size(sta_plan_t pl, size_t *fwd, size_t *bwd) {
+  if (!pl) return STA_ERR_INVALID_ARG;
+  if (fwd) *fwd = fwd_workspace(pl);
+  if (bwd) *bwd = bwd_workspace(pl);
+  return STA_OK;
+}
+
+sta_status sta_plan_geometry(sta_plan_t pl, int32_t *n_tiles, int32_t *tile_volume) {
+  if (!pl) return STA_ERR_INVALID_ARG;
+  if (n_tiles) *n_tiles = pl->g.n_tiles;
+  if (tile_volume) *tile_volume = pl->g.tau;
+  return STA_OK;
+}
+
+sta_status sta_plan_kv_tiles(sta_plan_t pl, int32_t head, int32_t *out, size_t cap, size_t *n) {
+  if (!pl || !n || head < 0 || head >= pl->g.Hh) return STA_ERR_INVALID_ARG;
+  const int per = pl->count[head];
+  *n = (size_t)pl->g.n_tiles * per;
+  if (!out) return STA_OK;
+  if (cap < *n) return STA_ERR_INVALID_ARG;
+  for (int q = 0; q < pl->g.n_tiles; ++q)
+    std::memcpy(out + (size_t)q * per, &pl->kv_list[((size_t)head * pl->g.n_tiles + q) * pl->kv_stride],
+                per * sizeof(int32_t));
+  return STA_OK;
+}
+
+sta_status sta_plan_q_tiles(sta_plan_t pl, int32_t head, int32_t *offsets, int32_t *indices, size_t cap,
+                            size_t *n_indices) {
+  if (!pl || head < 0 || head >= pl->g.Hh) return STA_ERR_INVALID_ARG;
+  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;  // plan built without STA_PROBLEM_BACKWARD
+  const int32_t *off = &pl->inv_off[(size_t)head * (pl->g.n_tiles + 1)];
+  const size_t n = (size_t)(off[pl->g.n_tiles] - off[0]);
+  if (n_indices) *n_indices = n;
+  if (offsets)
+    for (int k = 0; k <= pl->g.n_tiles; ++k) offsets[k] = off[k] - off[0];
+  if (indices) {
+    if (cap < n) return STA_ERR_INVALID_ARG;
+    std::memcpy(indices, &pl->inv_idx[off[0]], n * sizeof(int32_t));
+  }
+  return STA_OK;
+}
+
+sta_status sta_permute(sta_plan_t pl, const void *src, void *dst, int32_t inverse, void *stream) {
+  if (!pl || !src || !dst || pl->host_only) return STA_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return STA_ERR_ALIGNMENT;
+  const size_t bytes = tensor_bytes(pl);
+  const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
+  if (s < d + bytes && d < s + bytes) return STA_ERR_INVALID_ARG;
+  sta::PermuteParams pp{};
+  pp.g = pl->g;
+  pp.src = src;
+  pp.dst = dst;
+  pp.inverse = inverse ? 1 : 0;
+  if (sta::launch_permute(pp, pl->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return STA_ERR_CUDA;
+  return STA_OK;
+}
+
+sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *v, void *o, float *lse,
+                       void *workspace, size_t ws_bytes, void *stream_, uint32_t flags) {
+  if (!pl || !q || !k || !v || !o || pl->host_only) return STA_ERR_INVALID_ARG;
+  if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return STA_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < fwd_workspace(pl)) return STA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return STA_ERR_ALIGNMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char *ws = static_cast<char *>(workspace);
+  int *status = reinterpret_cast<int *>(ws);
+
+  const void *kbase = k, *vbase = v;
+  bool raster5d = pl->kv_mode == sta::kKvRaster5D;
+  if (!pl->tiled && !raster5d) {
+    // K and V are not readable as boxes: gather them tile-major first.
+    void *kt = ws + kStatusBytes, *vt = ws + kStatusBytes + tensor_bytes(pl);
+    sta::PermuteParams pp{};
+    pp.g = pl->g;
+    pp.inverse = 0;
+    pp.src = k, pp.dst = kt;
+    if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+    pp.src = v, pp.dst = vt;
+    if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+    kbase = kt, vbase = vt;
+  }
+  CUtensorMap mk, mv;
+  const bool ok = raster5d ? (make_map_5d(&mk, kbase, pl) && make_map_5d(&mv, vbase, pl))
+                           : (make_map_2d(&mk, kbase, pl) && make_map_2d(&mv, vbase, pl));
+  if (!ok) return STA_ERR_CUDA;
+
+  sta::FwdParams fp{};
+  fp.g = pl->g;
+  fp.q = q, fp.o = o, fp.lse = lse;
+  fp.tiled = pl->tiled ? 1 : 0;
+  fp.nqb = pl->nqb;
+  fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
+  fp.work = pl->d_work, fp.n_work = (int)pl->work.size();
+  fp.scale_log2 = pl->scale * 1.4426950408889634f;
+  fp.status = status;
+  fp.wait_limit_ns = g_wait_limit_ns;
+  fp.kv_mode = raster5d ? sta::kKvRaster5D : sta::kKvTiled2D;
+  fp.piece_rows = pl->piece_rows;
+  fp.box_w = pl->box_w, fp.box_h = pl->box_h, fp.box_t = pl->box_t;
+  fp.oob_coord = raster5d ? pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
+
+  if (flags & STA_CALL_CHECK)
+    if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;
+  if (sta::launch_forward(fp, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+  return finish_call(pl, workspace, stream, flags);
+}
+
+sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void *v, const void *o,
+                        const float *lse, const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                        size_t ws_bytes, void *stream, uint32_t flags) {
+  if (!pl || !q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || pl->host_only)
+    return STA_ERR_INVALID_ARG;
+  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;
+  (void)workspace, (void)ws_bytes, (void)stream, (void)flags;
+  return STA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

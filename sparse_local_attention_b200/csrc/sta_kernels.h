@@ -1,0 +1,67 @@
+// sta_kernels.h -- parameter blocks and launchers shared by the host API
+// (sta_api.cpp) and the CUDA kernels.  Internal to libsta.so.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace sta {
+
+// Status codes the kernels write into the workspace status word.
+enum KernelError : int {
+  kErrNone = 0,
+  kErrWaitProducer = 0x101,  // producer: waited too long for a free stage
+  kErrWaitMma = 0x102,       // MMA issuer: waited too long for data / softmax
+  kErrWaitSoftmax = 0x103,   // softmax warps: waited too long for an MMA result
+  kErrWaitEpilogue = 0x104,
+  kErrBwdWait = 0x201,
+};
+
+// How the K/V tiles are read by TMA.
+enum KvMode : int {
+  kKvTiled2D = 0,   // 2D map over a tile-major [B*Hh*N][d] buffer
+  kKvRaster5D = 1,  // 5D map (d, W, H, T, B*Hh) over the raster tensor
+};
+
+struct Geometry {
+  int B, Hh, d, N;
+  int T, H, W;
+  int tt, th, tw;
+  int GT, GH, GW;
+  int n_tiles, tau;  // tiles per (b, h) slice, tokens per tile
+};
+
+struct FwdParams {
+  Geometry g;
+  const void *q;     // bf16, token order given by `tiled`
+  void *o;           // bf16
+  float *lse;        // fp32, nullable
+  int tiled;         // q / o / lse are tile-major instead of raster
+  int nqb;           // query blocks of 128 rows per tile = ceil(tau / 128)
+  const int32_t *kv_list;   // [Hh][n_tiles][kv_stride]
+  const int32_t *kv_count;  // [Hh]
+  int kv_stride;
+  const int2 *work;  // (bh, tile * nqb + qblock), heaviest first
+  int n_work;
+  float scale_log2;  // softmax scale * log2(e)
+  int *status;       // device status word
+  unsigned long long wait_limit_ns;
+  // K/V gather geometry
+  int kv_mode;
+  int piece_rows;            // rows per TMA box (divides both tau and 128)
+  int box_w, box_h, box_t;   // 5D box extents in tokens
+  int oob_coord;             // coordinate past the end (zero-filled load)
+};
+
+struct PermuteParams {
+  Geometry g;
+  const void *src;
+  void *dst;
+  int inverse;
+};
+
+cudaError_t launch_forward(const FwdParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
+                           int num_sms, cudaStream_t stream);
+cudaError_t launch_permute(const PermuteParams &p, int num_sms, cudaStream_t stream);
+
+}  // namespace sta

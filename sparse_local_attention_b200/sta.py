@@ -1,0 +1,266 @@
+"""Python binding of libsta.so (ctypes).
+
+Argument marshalling only: every step of the attention path runs in the CUDA
+kernels behind the C ABI of include/sta.h.  PyTorch supplies device memory and
+the current stream.  There is no fallback: if the library cannot be loaded the
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import Optional, Sequence
+
+import torch
+
+from . import _build
+
+STA_OK = 0
+STATUS_NAMES = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_SHAPE", 3: "STA_ERR_UNSUPPORTED",
+                4: "STA_ERR_ALIGNMENT", 5: "STA_ERR_WORKSPACE", 6: "STA_ERR_OOM", 7: "STA_ERR_CUDA",
+                8: "STA_ERR_TIMEOUT"}
+STA_PROBLEM_BACKWARD = 0x1
+STA_PROBLEM_TILED = 0x2
+STA_PROBLEM_HOST_ONLY = 0x4
+STA_CALL_CHECK = 0x1
+
+EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
+            "sta_plan_q_tiles", "sta_plan_geometry", "sta_permute", "sta_forward", "sta_backward",
+            "sta_status_string", "sta_set_wait_limit_ns"]
+
+
+class StaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({status_string(status)})")
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("T", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("tile_t", ctypes.c_int32), ("tile_h", ctypes.c_int32), ("tile_w", ctypes.c_int32),
+                ("window", ctypes.POINTER(ctypes.c_int32)), ("scale", ctypes.c_float),
+                ("flags", ctypes.c_uint32)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsta.so (building it with nvcc first if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_build.LIB):
+        _build.build()
+    L = ctypes.CDLL(_build.LIB)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    szp = ctypes.POINTER(ctypes.c_size_t)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    L.sta_plan_create.argtypes = [ctypes.POINTER(_Problem), ctypes.POINTER(vp)]
+    L.sta_plan_destroy.argtypes = [vp]
+    L.sta_plan_workspace_size.argtypes = [vp, szp, szp]
+    L.sta_plan_kv_tiles.argtypes = [vp, ctypes.c_int32, i32p, sz, szp]
+    L.sta_plan_q_tiles.argtypes = [vp, ctypes.c_int32, i32p, i32p, sz, szp]
+    L.sta_plan_geometry.argtypes = [vp, i32p, i32p]
+    L.sta_permute.argtypes = [vp, vp, vp, ctypes.c_int32, vp]
+    L.sta_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
+    L.sta_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
+    L.sta_status_string.argtypes = [ctypes.c_int]
+    L.sta_status_string.restype = ctypes.c_char_p
+    L.sta_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.sta_set_wait_limit_ns.restype = None
+    for name in EXPORTED:
+        if name not in ("sta_status_string", "sta_set_wait_limit_ns"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().sta_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != STA_OK:
+        raise StaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+@dataclass
+class Problem:
+    batch: int
+    heads: int
+    head_dim: int
+    T: int
+    H: int
+    W: int
+    tile: tuple
+    windows: Sequence  # per head (w_t, w_h, w_w)
+    scale: float = 0.0
+    backward: bool = False
+    tiled: bool = False
+    host_only: bool = False
+
+    def _c(self):
+        flat = [int(x) for w in self.windows for x in w]
+        arr = (ctypes.c_int32 * max(1, len(flat)))(*flat)
+        flags = ((STA_PROBLEM_BACKWARD if self.backward else 0) | (STA_PROBLEM_TILED if self.tiled else 0)
+                 | (STA_PROBLEM_HOST_ONLY if self.host_only else 0))
+        p = _Problem(self.batch, self.heads, self.head_dim, self.T, self.H, self.W, *self.tile,
+                     ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), float(self.scale), flags)
+        return p, arr
+
+    @staticmethod
+    def from_workload(wl, backward=None, tiled=False, host_only=False, scale=0.0) -> "Problem":
+        return Problem(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows), scale,
+                       bool(wl.backward if backward is None else backward), tiled, host_only)
+
+
+class Plan:
+    """Owns an sta_plan_t.  Create with sta_plan_create()."""
+
+    def __init__(self, handle: ctypes.c_void_p, problem: Problem):
+        self.handle = handle
+        self.problem = problem
+        fwd, bwd = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().sta_plan_workspace_size(handle, ctypes.byref(fwd), ctypes.byref(bwd)), "sta_plan_workspace_size")
+        self.fwd_workspace_bytes = fwd.value
+        self.bwd_workspace_bytes = bwd.value
+        nt, tv = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().sta_plan_geometry(handle, ctypes.byref(nt), ctypes.byref(tv)), "sta_plan_geometry")
+        self.n_tiles, self.tile_volume = nt.value, tv.value
+
+    def destroy(self):
+        if self.handle is not None and self.handle.value:
+            _check(lib().sta_plan_destroy(self.handle), "sta_plan_destroy")
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+    def workspace(self, backward=False, device=None) -> torch.Tensor:
+        n = self.bwd_workspace_bytes if backward else self.fwd_workspace_bytes
+        return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sta_plan_create(problem: Problem) -> Plan:
+    cp, keep = problem._c()
+    h = ctypes.c_void_p()
+    _check(lib().sta_plan_create(ctypes.byref(cp), ctypes.byref(h)), "sta_plan_create")
+    del keep
+    return Plan(h, problem)
+
+
+def sta_plan_destroy(plan: Plan):
+    plan.destroy()
+
+
+def sta_plan_workspace_size(plan: Plan):
+    return plan.fwd_workspace_bytes, plan.bwd_workspace_bytes
+
+
+def sta_plan_kv_tiles(plan: Plan, head: int) -> torch.Tensor:
+    """[n_tiles, per_tile] int32 KV-tile lists of one head (host copy)."""
+    n = ctypes.c_size_t()
+    _check(lib().sta_plan_kv_tiles(plan.handle, head, None, 0, ctypes.byref(n)), "sta_plan_kv_tiles")
+    out = torch.empty(n.value, dtype=torch.int32)
+    _check(lib().sta_plan_kv_tiles(plan.handle, head, ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+                                   n.value, ctypes.byref(n)), "sta_plan_kv_tiles")
+    return out.view(plan.n_tiles, -1)
+
+
+def sta_plan_q_tiles(plan: Plan, head: int):
+    """(offsets[n_tiles + 1], indices) inverse lists of one head (host copy)."""
+    n = ctypes.c_size_t()
+    _check(lib().sta_plan_q_tiles(plan.handle, head, None, None, 0, ctypes.byref(n)), "sta_plan_q_tiles")
+    off = torch.empty(plan.n_tiles + 1, dtype=torch.int32)
+    idx = torch.empty(max(1, n.value), dtype=torch.int32)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    _check(lib().sta_plan_q_tiles(plan.handle, head, ctypes.cast(off.data_ptr(), i32p),
+                                  ctypes.cast(idx.data_ptr(), i32p), n.value, ctypes.byref(n)), "sta_plan_q_tiles")
+    return off, idx[: n.value]
+
+
+def sta_permute(plan: Plan, src: torch.Tensor, dst: Optional[torch.Tensor] = None, inverse: bool = False,
+                stream=None) -> torch.Tensor:
+    if dst is None:
+        dst = torch.empty_like(src)
+    _check(lib().sta_permute(plan.handle, _ptr(src), _ptr(dst), 1 if inverse else 0, _stream(stream)), "sta_permute")
+    return dst
+
+
+def _expect(t: torch.Tensor, name: str, shape, dtype):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} cuda={t.is_cuda}")
+
+
+def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                check: bool = False, want_lse: bool = True):
+    p = plan.problem
+    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _expect(t, nm, shape, torch.bfloat16)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:3], dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = plan.workspace(device=q.device)
+    st = lib().sta_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                           workspace.numel(), _stream(stream), STA_CALL_CHECK if check else 0)
+    _check(st, "sta_forward")
+    return o, lse
+
+
+def sta_backward(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, stream=None,
+                 check: bool = False):
+    p = plan.problem
+    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _expect(t, nm, shape, torch.bfloat16)
+    _expect(lse, "lse", shape[:3], torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = plan.workspace(backward=True, device=q.device)
+    st = lib().sta_backward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                            _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream),
+                            STA_CALL_CHECK if check else 0)
+    _check(st, "sta_backward")
+    return dq, dk, dv
+
+
+def sta_set_wait_limit_ns(ns: int):
+    lib().sta_set_wait_limit_ns(int(ns))
+
+
+def sliding_tile_attention(q, k, v, T, H, W, tile, windows, scale=0.0):
+    """One-shot convenience: plan + forward (the plan is rebuilt every call)."""
+    B, Hh, N, d = q.shape
+    plan = sta_plan_create(Problem(B, Hh, d, T, H, W, tuple(tile), tuple(tuple(w) for w in windows), scale))
+    try:
+        return sta_forward(plan, q, k, v)
+    finally:
+        torch.cuda.current_stream().synchronize()
+        plan.destroy()

@@ -1,0 +1,70 @@
+"""The C ABI loads, exports every symbol include/sta.h declares, and rejects
+bad arguments on the host (no GPU needed, no kernel launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_local_attention_b200 import sta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sta.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sta_[a-z_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    assert declared_functions() == sorted(sta.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(sta.library_path())
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in range(9):
+        assert sta.status_string(code)
+    assert sta.status_string(99) == "unknown status"
+
+
+def _create(**kw):
+    base = dict(batch=1, heads=1, head_dim=64, T=4, H=8, W=8, tile=(2, 4, 4), windows=[(1, 1, 1)], host_only=True)
+    base.update(kw)
+    return sta.sta_plan_create(sta.Problem(**base))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=5), 2),                      # tile does not divide T
+    (dict(tile=(3, 4, 4), T=6), 3),      # tile volume 48 ok? 48 % 8 == 0 -> fine below
+    (dict(head_dim=96), 3),
+    (dict(windows=[(0, 1, 1)]), 1),
+    (dict(batch=0), 2),
+    (dict(tile=(1, 1, 3), T=4, H=8, W=9), 3),  # tile volume 3, not a multiple of 8
+])
+def test_plan_rejects_bad_problems(kw, code):
+    if kw.get("tile") == (3, 4, 4):
+        _create(**kw)  # volume 48 is accepted
+        return
+    with pytest.raises(sta.StaError) as e:
+        _create(**kw)
+    assert e.value.status == code
+
+
+def test_compute_calls_on_host_only_plan_fail_cleanly():
+    plan = _create()
+    st = sta.lib().sta_forward(plan.handle, None, None, None, None, None, None, 0, None, 0)
+    assert st == 1
+    st = sta.lib().sta_permute(plan.handle, None, None, 0, None)
+    assert st == 1
+
+
+def test_backward_requires_backward_tables():
+    plan = _create()
+    with pytest.raises(sta.StaError):
+        sta.sta_plan_q_tiles(plan, 0)
