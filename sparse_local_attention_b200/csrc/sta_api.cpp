@@ -30,7 +30,7 @@ struct sta_plan_s {
   std::vector<int32_t> inv_idx;
   std::vector<int2> work;        // forward work items
   int nqb = 1;
-  int kv_mode = sta::kKvTiled2D;
+  int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
   bool host_only = false;
   bool tiled = false;
@@ -64,7 +64,7 @@ constexpr size_t kStatusBytes = 256;
 
 size_t fwd_workspace(const sta_plan_s *pl) {
   size_t b = kStatusBytes;
-  if (!pl->tiled && pl->kv_mode == sta::kKvTiled2D) b += 2 * tensor_bytes(pl);
+  if (!pl->tiled && pl->kv_mode == sta::kKvTiled) b += 2 * tensor_bytes(pl);
   return b;
 }
 
@@ -90,32 +90,41 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D map over a tile-major [rows][d] bf16 buffer, box 64 x piece_rows, 128B swizzle.
-bool make_map_2d(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+// Panels per TMA box: both 64-column panels of a 128-row chunk in one box
+// when the chunk is a single piece and d = 128; otherwise one panel per box.
+int box_panels(const sta_plan_s *pl) { return (pl->g.d == 128 && pl->piece_rows == 128) ? 2 : 1; }
+
+// Tile-major buffer [rows][d] bf16: (64, rows[, 2 panels]), box (64, piece_rows[, panels]).
+bool make_map_tiled(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const Geometry &g = pl->g;
-  cuuint64_t dims[2] = {(cuuint64_t)g.d, (cuuint64_t)g.B * g.Hh * g.N};
-  cuuint64_t strides[1] = {(cuuint64_t)g.d * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)pl->piece_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+  const cuuint64_t rows = (cuuint64_t)g.B * g.Hh * g.N;
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {(cuuint64_t)g.d * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)pl->piece_rows, (cuuint32_t)box_panels(pl)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const cuuint32_t rank = g.d == 128 ? 3 : 2;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 5D map (d, W, H, T, B*Hh) over a raster tensor; one box = one piece of a tile.
-bool make_map_5d(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+// Raster tensor: (64, W, H, T*B*Hh[, 2 panels]); one box = one piece of a tile
+// (whole w-runs and h-planes), so K/V tiles are gathered straight from the
+// raster layout with no permutation pass.
+bool make_map_raster(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const Geometry &g = pl->g;
   const cuuint64_t row = (cuuint64_t)g.d * 2;
-  cuuint64_t dims[5] = {(cuuint64_t)g.d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T,
-                        (cuuint64_t)g.B * g.Hh};
-  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * (cuuint64_t)g.N};
-  cuuint32_t box[5] = {64, (cuuint32_t)pl->box_w, (cuuint32_t)pl->box_h, (cuuint32_t)pl->box_t, 1};
+  cuuint64_t dims[5] = {64, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T * g.B * g.Hh, 2};
+  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, 128};
+  cuuint32_t box[5] = {64, (cuuint32_t)pl->box_w, (cuuint32_t)pl->box_h, (cuuint32_t)pl->box_t,
+                       (cuuint32_t)box_panels(pl)};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+  const cuuint32_t rank = g.d == 128 ? 5 : 4;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -304,11 +313,11 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
   // --- how K/V tiles reach shared memory
   pl->piece_rows = gcd_int(g.tau, 128);
   if (pl->tiled) {
-    pl->kv_mode = sta::kKvTiled2D;
+    pl->kv_mode = sta::kKvTiled;
   } else if (raster_box(g, pl->piece_rows, &pl->box_w, &pl->box_h, &pl->box_t)) {
-    pl->kv_mode = sta::kKvRaster5D;
+    pl->kv_mode = sta::kKvRaster;
   } else {
-    pl->kv_mode = sta::kKvTiled2D;  // permute K and V into the workspace first
+    pl->kv_mode = sta::kKvTiled;  // permute K and V into the workspace first
   }
 
   if (!pl->host_only) {
@@ -417,7 +426,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   int *status = reinterpret_cast<int *>(ws);
 
   const void *kbase = k, *vbase = v;
-  bool raster5d = pl->kv_mode == sta::kKvRaster5D;
+  bool raster5d = pl->kv_mode == sta::kKvRaster;
   if (!pl->tiled && !raster5d) {
     // K and V are not readable as boxes: gather them tile-major first.
     void *kt = ws + kStatusBytes, *vt = ws + kStatusBytes + tensor_bytes(pl);
@@ -431,8 +440,8 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
     kbase = kt, vbase = vt;
   }
   CUtensorMap mk, mv;
-  const bool ok = raster5d ? (make_map_5d(&mk, kbase, pl) && make_map_5d(&mv, vbase, pl))
-                           : (make_map_2d(&mk, kbase, pl) && make_map_2d(&mv, vbase, pl));
+  const bool ok = raster5d ? (make_map_raster(&mk, kbase, pl) && make_map_raster(&mv, vbase, pl))
+                           : (make_map_tiled(&mk, kbase, pl) && make_map_tiled(&mv, vbase, pl));
   if (!ok) return STA_ERR_CUDA;
 
   sta::FwdParams fp{};
@@ -445,10 +454,11 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   fp.scale_log2 = pl->scale * 1.4426950408889634f;
   fp.status = status;
   fp.wait_limit_ns = g_wait_limit_ns;
-  fp.kv_mode = raster5d ? sta::kKvRaster5D : sta::kKvTiled2D;
+  fp.kv_mode = raster5d ? sta::kKvRaster : sta::kKvTiled;
   fp.piece_rows = pl->piece_rows;
   fp.box_w = pl->box_w, fp.box_h = pl->box_h, fp.box_t = pl->box_t;
-  fp.oob_coord = raster5d ? pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
+  fp.box_panels = box_panels(pl);
+  fp.oob_coord = raster5d ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
 
   if (flags & STA_CALL_CHECK)
     if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;

@@ -18,9 +18,12 @@ enum KernelError : int {
 };
 
 // How the K/V tiles are read by TMA.
+// Both maps split the head dimension into 64-element (128-byte) panels; for
+// d = 128 the panel index is the outermost map dimension, so one box can
+// bring both panels of a chunk in a single TMA instruction.
 enum KvMode : int {
-  kKvTiled2D = 0,   // 2D map over a tile-major [B*Hh*N][d] buffer
-  kKvRaster5D = 1,  // 5D map (d, W, H, T, B*Hh) over the raster tensor
+  kKvTiled = 0,   // (64, B*Hh*N rows[, 2 panels]) over a tile-major buffer
+  kKvRaster = 1,  // (64, W, H, T*B*Hh[, 2 panels]) over the raster tensor
 };
 
 struct Geometry {
@@ -49,8 +52,9 @@ struct FwdParams {
   // K/V gather geometry
   int kv_mode;
   int piece_rows;            // rows per TMA box (divides both tau and 128)
-  int box_w, box_h, box_t;   // 5D box extents in tokens
-  int oob_coord;             // coordinate past the end (zero-filled load)
+  int box_w, box_h, box_t;   // raster box extents in tokens
+  int box_panels;            // panels per box: 2 = whole chunk row in one instruction
+  int oob_coord;             // row (tiled) or T*B*Hh (raster) coordinate past the end
 };
 
 struct PermuteParams {
