@@ -29,7 +29,7 @@ struct sta_plan_s {
   std::vector<int32_t> inv_off;  // [heads][n_tiles + 1], absolute into inv_idx
   std::vector<int32_t> inv_idx;
   std::vector<int2> work;        // forward work items
-  int nqb = 1;
+  int npairs = 1;
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
   bool host_only = false;
@@ -64,7 +64,7 @@ constexpr size_t kStatusBytes = 256;
 
 size_t fwd_workspace(const sta_plan_s *pl) {
   size_t b = kStatusBytes;
-  if (!pl->tiled && pl->kv_mode == sta::kKvTiled) b += 2 * tensor_bytes(pl);
+  if (!pl->tiled && pl->kv_mode == sta::kKvTiled) b += 3 * tensor_bytes(pl);
   return b;
 }
 
@@ -239,7 +239,7 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
   g.n_tiles = g.GT * g.GH * g.GW;
   g.tau = (int)tau;
   pl->scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt((float)g.d);
-  pl->nqb = (g.tau + 127) / 128;
+  pl->npairs = (g.tau + 255) / 256;
 
   try {
     // --- per-head clamped windows and list lengths
@@ -295,16 +295,23 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       }
     }
 
-    // --- forward work items, heaviest heads first (longest-processing-time
-    //     order for the persistent grid); within a head, (batch, tile, block)
+    // --- forward work items: pairs of 128-row query blocks of one tile.
+    //     Heaviest heads first (longest-processing-time order for the
+    //     persistent grid); within a head, the two-block items before the
+    //     one-block tail items of tiles with an odd block count.
     std::vector<int> heads(g.Hh);
     std::iota(heads.begin(), heads.end(), 0);
     std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
-    pl->work.reserve((size_t)g.B * g.Hh * g.n_tiles * pl->nqb);
+    const int nqb = (g.tau + 127) / 128;
+    pl->work.reserve((size_t)g.B * g.Hh * g.n_tiles * pl->npairs);
     for (int h : heads)
       for (int b = 0; b < g.B; ++b)
-        for (int t = 0; t < g.n_tiles; ++t)
-          for (int qb = 0; qb < pl->nqb; ++qb) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->nqb + qb));
+        for (int full_pair = 1; full_pair >= 0; --full_pair)
+          for (int t = 0; t < g.n_tiles; ++t)
+            for (int pr = 0; pr < pl->npairs; ++pr) {
+              const bool has_b = 2 * pr + 1 < nqb;
+              if (has_b == (full_pair == 1)) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
+            }
   } catch (const std::bad_alloc &) {
     delete pl;
     return STA_ERR_OOM;
@@ -425,30 +432,35 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   char *ws = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(ws);
 
-  const void *kbase = k, *vbase = v;
+  const void *qbase = q, *kbase = k, *vbase = v;
   bool raster5d = pl->kv_mode == sta::kKvRaster;
   if (!pl->tiled && !raster5d) {
-    // K and V are not readable as boxes: gather them tile-major first.
-    void *kt = ws + kStatusBytes, *vt = ws + kStatusBytes + tensor_bytes(pl);
-    sta::PermuteParams pp{};
-    pp.g = pl->g;
-    pp.inverse = 0;
-    pp.src = k, pp.dst = kt;
-    if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
-    pp.src = v, pp.dst = vt;
-    if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
-    kbase = kt, vbase = vt;
+    // Tiles are not readable as TMA boxes of the raster tensor: gather Q, K
+    // and V tile-major into the workspace first.
+    char *dst = ws + kStatusBytes;
+    const void *src[3] = {q, k, v};
+    const void **base[3] = {&qbase, &kbase, &vbase};
+    for (int i = 0; i < 3; ++i) {
+      sta::PermuteParams pp{};
+      pp.g = pl->g;
+      pp.inverse = 0;
+      pp.src = src[i], pp.dst = dst + i * tensor_bytes(pl);
+      if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+      *base[i] = pp.dst;
+    }
   }
-  CUtensorMap mk, mv;
-  const bool ok = raster5d ? (make_map_raster(&mk, kbase, pl) && make_map_raster(&mv, vbase, pl))
-                           : (make_map_tiled(&mk, kbase, pl) && make_map_tiled(&mv, vbase, pl));
+  CUtensorMap mq, mk, mv;
+  const bool ok = raster5d ? (make_map_raster(&mq, qbase, pl) && make_map_raster(&mk, kbase, pl) &&
+                              make_map_raster(&mv, vbase, pl))
+                           : (make_map_tiled(&mq, qbase, pl) && make_map_tiled(&mk, kbase, pl) &&
+                              make_map_tiled(&mv, vbase, pl));
   if (!ok) return STA_ERR_CUDA;
 
   sta::FwdParams fp{};
   fp.g = pl->g;
   fp.q = q, fp.o = o, fp.lse = lse;
   fp.tiled = pl->tiled ? 1 : 0;
-  fp.nqb = pl->nqb;
+  fp.npairs = pl->npairs;
   fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
   fp.work = pl->d_work, fp.n_work = (int)pl->work.size();
   fp.scale_log2 = pl->scale * 1.4426950408889634f;
@@ -462,7 +474,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
 
   if (flags & STA_CALL_CHECK)
     if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;
-  if (sta::launch_forward(fp, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+  if (sta::launch_forward(fp, mq, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
   return finish_call(pl, workspace, stream, flags);
 }
 

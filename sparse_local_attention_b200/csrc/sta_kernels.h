@@ -40,11 +40,11 @@ struct FwdParams {
   void *o;           // bf16
   float *lse;        // fp32, nullable
   int tiled;         // q / o / lse are tile-major instead of raster
-  int nqb;           // query blocks of 128 rows per tile = ceil(tau / 128)
+  int npairs;        // work items per tile: pairs of 128-row query blocks = ceil(tau / 256)
   const int32_t *kv_list;   // [Hh][n_tiles][kv_stride]
   const int32_t *kv_count;  // [Hh]
   int kv_stride;
-  const int2 *work;  // (bh, tile * nqb + qblock), heaviest first
+  const int2 *work;  // (bh, tile * npairs + pair), heaviest first
   int n_work;
   float scale_log2;  // softmax scale * log2(e)
   int *status;       // device status word
@@ -64,8 +64,8 @@ struct PermuteParams {
   int inverse;
 };
 
-cudaError_t launch_forward(const FwdParams &p, const CUtensorMap &tmap_k, const CUtensorMap &tmap_v,
-                           int num_sms, cudaStream_t stream);
+cudaError_t launch_forward(const FwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                           const CUtensorMap &tmap_v, int num_sms, cudaStream_t stream);
 cudaError_t launch_permute(const PermuteParams &p, int num_sms, cudaStream_t stream);
 
 }  // namespace sta
