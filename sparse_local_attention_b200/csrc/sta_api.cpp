@@ -297,21 +297,16 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
 
     // --- forward work items: pairs of 128-row query blocks of one tile.
     //     Heaviest heads first (longest-processing-time order for the
-    //     persistent grid); within a head, the two-block items before the
-    //     one-block tail items of tiles with an odd block count.
+    //     persistent grid); within a head, tile by tile, so consecutive items
+    //     share most of their key tiles in L2.
     std::vector<int> heads(g.Hh);
     std::iota(heads.begin(), heads.end(), 0);
     std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
-    const int nqb = (g.tau + 127) / 128;
     pl->work.reserve((size_t)g.B * g.Hh * g.n_tiles * pl->npairs);
     for (int h : heads)
       for (int b = 0; b < g.B; ++b)
-        for (int full_pair = 1; full_pair >= 0; --full_pair)
-          for (int t = 0; t < g.n_tiles; ++t)
-            for (int pr = 0; pr < pl->npairs; ++pr) {
-              const bool has_b = 2 * pr + 1 < nqb;
-              if (has_b == (full_pair == 1)) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
-            }
+        for (int t = 0; t < g.n_tiles; ++t)
+          for (int pr = 0; pr < pl->npairs; ++pr) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
   } catch (const std::bad_alloc &) {
     delete pl;
     return STA_ERR_OOM;

@@ -25,8 +25,8 @@
 //   * warps 0-3 / 4-7: softmax of block A / B.  Query row r lives in TMEM lane
 //     r and a thread owns one whole row: row max and sum need no shuffles.
 //     fp32 online softmax in the log2 domain with lazy rescaling of O (only
-//     when the running max grows by more than 2^8); P is rounded to bf16 on
-//     the integer pipe so the XU pipe only runs ex2.
+//     when the running max grows by more than 2^8).  ex2 runs on the XU pipe,
+//     the bf16 packing (cvt) on another, so they overlap.
 //   * Tensor memory (512 columns): S_A/P_A [0,128) S_B/P_B [128,256)
 //     O_A [256,256+d) O_B [256+d,256+2d).
 // Every barrier wait is bounded; on a time-out the kernel records an error in
@@ -259,25 +259,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t p_waits[2] = {0, 0}, o_waits[2] = {0, 0}, x_items[2] = {0, 0};
       bool ok = true, issued = false;
 
+      // Shared-memory descriptors are built once; a k-step only adds to the
+      // start-address field (bits 0..13, address >> 4), which cannot carry
+      // because every operand lies below 256 KB.
+      const uint64_t qdesc0 = smem_desc_sw128(q_addr, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(slots_addr, 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(slots_addr, C::kPanelBytes, 1024);
       // S_X = Q_X K^T for the K chunk in ring slot `slot`.
       auto mma_s = [&](int x, uint32_t slot) {
-        const uint32_t kbase = slots_addr + slot * C::kTileBytes, qbase = q_addr + x * C::kTileBytes;
+        const uint64_t qd = qdesc0 + ((x * C::kTileBytes) >> 4), kd = kdesc0 + ((slot * C::kTileBytes) >> 4);
+        const uint32_t d_tm = tmem + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kPanelBytes + (kk % 4) * 32;
-          mma_ss(tmem + 128 * x, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * C::kPanelBytes + (kk % 4) * 32) >> 4;
+          mma_ss(d_tm, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[x]);
       };
       // O_X += P_X V for the V chunk in ring slot `slot`.
       auto mma_pv = [&](int x, uint32_t slot, bool first) {
-        const uint32_t vbase = slots_addr + slot * C::kTileBytes;
+        const uint64_t vd = vdesc0 + ((slot * C::kTileBytes) >> 4);
+        const uint32_t o_tm = tmem + C::kTmO0 + x * D, p_tm = tmem + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + C::kTmO0 + x * D, tmem + 128 * x + kk * 8,
-                 smem_desc_sw128(vbase + kk * 16 * 128, C::kPanelBytes, 1024), idesc_pv,
-                 (first && kk == 0) ? 0u : 1u);
+          mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
         mma_commit(&pv_done[x]);
       };
       auto wait_slot = [&](uint32_t slot_ld) -> bool {
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float p0 = ex2_approx(fmaf(s[32 * c + i], sl2, -m));
             const float p1 = ex2_approx(fmaf(s[32 * c + i + 1], sl2, -m));
             ls[(i / 2) & 7] += p0 + p1;
-            pk[i / 2] = pack_bf16_rna(p0, p1);
+            pk[i / 2] = pack_bf16(p0, p1);
           }
           tmem_st16(tmem + lane_off + s_col + c * 16, pk);
         }
