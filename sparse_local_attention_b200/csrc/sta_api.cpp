@@ -29,6 +29,8 @@ struct sta_plan_s {
   std::vector<int32_t> inv_off;  // [heads][n_tiles + 1], absolute into inv_idx
   std::vector<int32_t> inv_idx;
   std::vector<int2> work;        // forward work items
+  std::vector<int2> work_kv;     // backward dK/dV items (bh, key tile * nqb + key block)
+  std::vector<int2> work_q;      // backward dQ items (bh, query tile * nqb + query block)
   int npairs = 1;
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
@@ -38,7 +40,7 @@ struct sta_plan_s {
   int device = -1, num_sms = 0;
   // device copies
   int32_t *d_kv_list = nullptr, *d_count = nullptr, *d_inv_off = nullptr, *d_inv_idx = nullptr;
-  int2 *d_work = nullptr;
+  int2 *d_work = nullptr, *d_work_kv = nullptr, *d_work_q = nullptr;
 };
 
 namespace {
@@ -68,8 +70,17 @@ size_t fwd_workspace(const sta_plan_s *pl) {
   return b;
 }
 
+// Backward workspace: status word, then LSE*log2(e) and D = rowsum(dO*O),
+// tile-major with a pitch of N + 128 floats per (batch, head) slice, then (only
+// when tiles are not readable as boxes of the raster tensors) tile-major
+// copies of Q, K, V and dO.
+size_t lse_pitch_bytes(const sta_plan_s *pl) { return ((size_t)pl->g.N + 128) * 4; }
+size_t bwd_vec_bytes(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * lse_pitch_bytes(pl); }
 size_t bwd_workspace(const sta_plan_s *pl) {
-  return kStatusBytes;
+  size_t b = kStatusBytes + 2 * bwd_vec_bytes(pl);
+  b = (b + 255) & ~size_t(255);
+  if (!pl->tiled && pl->kv_mode == sta::kKvTiled) b += 4 * tensor_bytes(pl);
+  return b;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -135,8 +146,10 @@ void free_device(sta_plan_s *pl) {
   cudaFree(pl->d_inv_off);
   cudaFree(pl->d_inv_idx);
   cudaFree(pl->d_work);
+  cudaFree(pl->d_work_kv);
+  cudaFree(pl->d_work_q);
   pl->d_kv_list = pl->d_count = pl->d_inv_off = pl->d_inv_idx = nullptr;
-  pl->d_work = nullptr;
+  pl->d_work = pl->d_work_kv = pl->d_work_q = nullptr;
 }
 
 template <class T>
@@ -307,6 +320,27 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       for (int b = 0; b < g.B; ++b)
         for (int t = 0; t < g.n_tiles; ++t)
           for (int pr = 0; pr < pl->npairs; ++pr) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
+
+    if (prob->flags & STA_PROBLEM_BACKWARD) {
+      const int nqb = (g.tau + 127) / 128;
+      // dQ: one 128-row query block per item, heaviest heads first.
+      for (int h : heads)
+        for (int b = 0; b < g.B; ++b)
+          for (int t = 0; t < g.n_tiles; ++t)
+            for (int qb = 0; qb < nqb; ++qb) pl->work_q.push_back(make_int2(b * g.Hh + h, t * nqb + qb));
+      // dK/dV: one 128-row key block per item, longest inverse list first.
+      struct KvItem { int len, bh, key; };
+      std::vector<KvItem> items;
+      items.reserve((size_t)g.B * g.Hh * g.n_tiles * nqb);
+      for (int h = 0; h < g.Hh; ++h)
+        for (int b = 0; b < g.B; ++b)
+          for (int t = 0; t < g.n_tiles; ++t) {
+            const int32_t *off = &pl->inv_off[(size_t)h * (g.n_tiles + 1) + t];
+            for (int kb = 0; kb < nqb; ++kb) items.push_back({off[1] - off[0], b * g.Hh + h, t * nqb + kb});
+          }
+      std::stable_sort(items.begin(), items.end(), [](const KvItem &a, const KvItem &c) { return a.len > c.len; });
+      for (const KvItem &it : items) pl->work_kv.push_back(make_int2(it.bh, it.key));
+    }
   } catch (const std::bad_alloc &) {
     delete pl;
     return STA_ERR_OOM;
@@ -339,7 +373,8 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     pl->device = dev;
     std::vector<int32_t> cnt(pl->count);
     if (!upload(&pl->d_kv_list, pl->kv_list) || !upload(&pl->d_count, cnt) || !upload(&pl->d_work, pl->work) ||
-        !upload(&pl->d_inv_off, pl->inv_off) || !upload(&pl->d_inv_idx, pl->inv_idx)) {
+        !upload(&pl->d_inv_off, pl->inv_off) || !upload(&pl->d_inv_idx, pl->inv_idx) ||
+        !upload(&pl->d_work_kv, pl->work_kv) || !upload(&pl->d_work_q, pl->work_q)) {
       cudaError_t e = cudaGetLastError();
       free_device(pl);
       delete pl;
@@ -475,12 +510,66 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
 
 sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void *v, const void *o,
                         const float *lse, const void *dout, void *dq, void *dk, void *dv, void *workspace,
-                        size_t ws_bytes, void *stream, uint32_t flags) {
+                        size_t ws_bytes, void *stream_, uint32_t flags) {
   if (!pl || !q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || pl->host_only)
     return STA_ERR_INVALID_ARG;
-  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;
-  (void)workspace, (void)ws_bytes, (void)stream, (void)flags;
-  return STA_ERR_UNSUPPORTED;
+  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;  // plan built without STA_PROBLEM_BACKWARD
+  if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  const void *ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return STA_ERR_ALIGNMENT;
+  if (ws_bytes < bwd_workspace(pl)) return STA_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char *ws = static_cast<char *>(workspace);
+  int *status = reinterpret_cast<int *>(ws);
+  float *lse2_t = reinterpret_cast<float *>(ws + kStatusBytes);
+  float *dd_t = reinterpret_cast<float *>(ws + kStatusBytes + bwd_vec_bytes(pl));
+
+  const void *base[4] = {q, k, v, dout};
+  const bool raster = pl->kv_mode == sta::kKvRaster;
+  if (!pl->tiled && !raster) {
+    char *dst = ws + ((kStatusBytes + 2 * bwd_vec_bytes(pl) + 255) & ~size_t(255));
+    for (int i = 0; i < 4; ++i) {
+      sta::PermuteParams pp{};
+      pp.g = pl->g;
+      pp.inverse = 0;
+      pp.src = base[i], pp.dst = dst + i * tensor_bytes(pl);
+      if (sta::launch_permute(pp, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+      base[i] = pp.dst;
+    }
+  }
+  CUtensorMap maps[4];
+  for (int i = 0; i < 4; ++i) {
+    const bool ok = raster ? make_map_raster(&maps[i], base[i], pl) : make_map_tiled(&maps[i], base[i], pl);
+    if (!ok) return STA_ERR_CUDA;
+  }
+
+  sta::BwdParams bp{};
+  bp.g = pl->g;
+  bp.tiled = pl->tiled ? 1 : 0;
+  bp.nqb = (pl->g.tau + 127) / 128;
+  bp.kv_mode = raster ? sta::kKvRaster : sta::kKvTiled;
+  bp.piece_rows = pl->piece_rows;
+  bp.box_w = pl->box_w, bp.box_h = pl->box_h, bp.box_t = pl->box_t;
+  bp.box_panels = box_panels(pl);
+  bp.oob_coord = raster ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
+  bp.o = o, bp.dout = dout, bp.lse = lse;
+  bp.lse2_t = lse2_t, bp.dd_t = dd_t;
+  bp.dq = dq, bp.dk = dk, bp.dv = dv;
+  bp.kv_list = pl->d_kv_list, bp.kv_count = pl->d_count, bp.kv_stride = pl->kv_stride;
+  bp.inv_off = pl->d_inv_off, bp.inv_idx = pl->d_inv_idx;
+  bp.work_kv = pl->d_work_kv, bp.n_work_kv = (int)pl->work_kv.size();
+  bp.work_q = pl->d_work_q, bp.n_work_q = (int)pl->work_q.size();
+  bp.scale = pl->scale;
+  bp.scale_log2 = pl->scale * 1.4426950408889634f;
+  bp.status = status;
+  bp.wait_limit_ns = g_wait_limit_ns;
+
+  if (flags & STA_CALL_CHECK)
+    if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;
+  if (sta::launch_backward(bp, maps[0], maps[1], maps[2], maps[3], pl->num_sms, stream) != cudaSuccess)
+    return STA_ERR_CUDA;
+  return finish_call(pl, workspace, stream, flags);
 }
 
 }  // extern "C"

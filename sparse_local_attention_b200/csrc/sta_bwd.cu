@@ -1,0 +1,640 @@
+// sta_bwd.cu -- Sliding Tile Attention backward kernels for sm_100a.
+//
+// Gradients of the windowed attention ("Fast Video Generation with Sliding
+// Tile Attention", Abstract: fine-tuning with STA).  With P = softmax of the
+// scores inside each query's window (recomputed from the forward LSE) and
+// D_i = sum_c dO_ic O_ic:
+//   dV = P^T dO,  dS = P o (dO V^T - D),  dK = scale dS^T Q,  dQ = scale dS K,
+// every sum running only over the (query, key) pairs of the window.
+//
+// Three launches, no atomics (the result is deterministic):
+//   1. bwd_pre: D and LSE * log2(e) per query row, stored tile-major so a
+//      128-row block reads them as one contiguous run.
+//   2. bwd_dkdv: one 128-row key block per work item (key-block major).  K and
+//      V stay in shared memory; the query blocks of every query tile whose
+//      window holds the key tile (the planner's inverse lists) stream through
+//      a ring.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the softmax warps
+//      (thread = key row) turn them into P^T and dS^T (bf16, written over the
+//      consumed columns), then dV += P^T dO and dK += dS^T Q accumulate in
+//      TMEM with P^T / dS^T as the TMEM A operand.
+//   3. bwd_dq: one 128-row query block per work item (query-block major, the
+//      forward KV-tile lists).  S = Q K^T and dP = dO V^T per 128-key chunk,
+//      dS in TMEM, dQ += dS K.
+// Warp roles as in the forward: warps 0-3 elementwise math (thread = TMEM
+// lane = row), warp 4 TMA producer, warp 5 MMA issuer.  Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+#include "sta_common.cuh"
+#include "sta_kernels.h"
+
+namespace sta {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr int kMaxCoords = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ long long lse_pitch(const Geometry &g) { return (long long)g.N + 128; }
+
+// ----------------------------------------------------------------------- 1. preprocess
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
+  const Geometry &g = p.g;
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)g.B * g.Hh * g.N;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < nrows; r += warps) {
+    const int bh = (int)(r / g.N), pos = (int)(r - (long long)bh * g.N);
+    const int tile = pos / g.tau, o = pos - tile * g.tau;
+    const long long tok = token_row(g, p.tiled, bh, tile, o);
+    const __nv_bfloat16 *orow = static_cast<const __nv_bfloat16 *>(p.o) + tok * D;
+    const __nv_bfloat16 *drow = static_cast<const __nv_bfloat16 *>(p.dout) + tok * D;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < D / 64; ++e) {
+      const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162 *>(orow)[lane + 32 * e];
+      const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162 *>(drow)[lane + 32 * e];
+      const float2 af = __bfloat1622float2(a), bf = __bfloat1622float2(b);
+      acc = fmaf(af.x, bf.x, fmaf(af.y, bf.y, acc));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+      const long long dst = bh * lse_pitch(g) + pos;
+      p.dd_t[dst] = acc;
+      p.lse2_t[dst] = p.lse[tok] * kLog2e;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------- 2. dK, dV
+template <int D>
+struct DkvCfg {
+  static constexpr uint32_t kTile = kBM * D * 2;           // one 128-row operand tile
+  static constexpr uint32_t kPanel = kBM * 128;
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr uint32_t kStage = 2 * kTile + 1024;     // Q, dO, LSE2[128], D[128]
+  static constexpr int kNumBars = 2 * kStages + 7;
+  static constexpr uint32_t kSmem = 2 * kTile + kStages * kStage + kNumBars * 8 + 64 + 1024;
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 256 + D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
+                    const BwdParams p) {
+  using C = DkvCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *k_s = smem, *v_s = smem + C::kTile;
+  uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, lse2[128], dd[128]}
+  uint64_t *bars = reinterpret_cast<uint64_t *>(stages + C::kStages * C::kStage);
+  uint64_t *st_full = bars, *st_empty = bars + C::kStages;
+  uint64_t *kv_full = bars + 2 * C::kStages, *kv_free = kv_full + 1, *s_full = kv_full + 2, *p_ready = kv_full + 3;
+  uint64_t *acc_done = kv_full + 4, *acc_free = kv_full + 5, *drain = kv_full + 6;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Geometry &g = p.g;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&st_full[i], 1);
+      mbar_init(&st_empty[i], 1);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(kv_free, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, 4);
+    mbar_init(acc_done, 1);
+    mbar_init(acc_free, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+  const int pieces = kBM / p.piece_rows;
+
+  auto item_info = [&](int item, int &bh, int &ktile, int &kb, int &off0, int &nq) {
+    const int2 wi = p.work_kv[item];
+    bh = wi.x, ktile = wi.y / p.nqb, kb = wi.y % p.nqb;
+    const int32_t *io = p.inv_off + (long long)(bh % g.Hh) * (g.n_tiles + 1) + ktile;
+    off0 = io[0];
+    nq = (io[1] - io[0]) * p.nqb;
+  };
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      tma_prefetch_desc(&tmap_do);
+      uint32_t ld = 0, item_ctr = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
+        int bh, ktile, kb, off0, nq;
+        item_info(item, bh, ktile, kb, off0, nq);
+        if (!mbar_wait(kv_free, (item_ctr & 1) ^ 1, ctl, kErrBwdWait)) { ok = false; break; }
+        mbar_arrive_expect_tx(kv_full, 2 * C::kTile);
+        for (int pc = 0; pc < pieces; ++pc) {
+          const int off = kb * kBM + pc * p.piece_rows;
+          const int4 c = box_coords(p, bh, ktile, off, off < g.tau);
+          load_box<D>(p, &tmap_k, k_s + pc * p.piece_rows * 128, c, kv_full);
+          load_box<D>(p, &tmap_v, v_s + pc * p.piece_rows * 128, c, kv_full);
+        }
+        for (int i = 0; i < nq && ok; ++i) {
+          const int qt = p.inv_idx[off0 + i / p.nqb], qb = i % p.nqb;
+          const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
+          if (!mbar_wait(&st_empty[st], ph ^ 1, ctl, kErrBwdWait)) { ok = false; break; }
+          uint8_t *sb = stages + st * C::kStage;
+          mbar_arrive_expect_tx(&st_full[st], C::kStage);
+          for (int pc = 0; pc < pieces; ++pc) {
+            const int off = qb * kBM + pc * p.piece_rows;
+            const int4 c = box_coords(p, bh, qt, off, off < g.tau);
+            load_box<D>(p, &tmap_q, sb + pc * p.piece_rows * 128, c, &st_full[st]);
+            load_box<D>(p, &tmap_do, sb + C::kTile + pc * p.piece_rows * 128, c, &st_full[st]);
+          }
+          const long long lo = bh * lse_pitch(g) + (long long)qt * g.tau + qb * kBM;
+          bulk_load(sb + 2 * C::kTile, p.lse2_t + lo, 512, &st_full[st]);
+          bulk_load(sb + 2 * C::kTile + 512, p.dd_t + lo, 512, &st_full[st]);
+          ++ld;
+        }
+        ++item_ctr;
+      }
+      if (!ok) {
+        const uint32_t first = ld > (uint32_t)C::kStages ? ld - C::kStages : 0;
+        for (uint32_t i = first; i < ld; ++i) drain_wait(&st_full[i % C::kStages], (i / C::kStages) & 1);
+        if (item_ctr > 0) drain_wait(kv_full, (item_ctr - 1) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(kBM, D, false, true);
+      const uint64_t kd = smem_desc_sw128(smem_u32(k_s), 16, 1024), vd = smem_desc_sw128(smem_u32(v_s), 16, 1024);
+      const uint64_t sk0 = smem_desc_sw128(smem_u32(stages), 16, 1024);              // K-major Q / dO
+      const uint64_t sm0 = smem_desc_sw128(smem_u32(stages), C::kPanel, 1024);       // MN-major Q / dO
+      uint32_t ld = 0, item_ctr = 0, p_waits = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
+        int bh, ktile, kb, off0, nq;
+        item_info(item, bh, ktile, kb, off0, nq);
+        if (!mbar_wait(kv_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
+        tc_fence_after();
+        for (int i = 0; i < nq && ok; ++i) {
+          const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
+          if (!mbar_wait(&st_full[st], ph, ctl, kErrBwdWait)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t so = (st * C::kStage) >> 4, dso = (st * C::kStage + C::kTile) >> 4;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit(s_full);
+          if (i == nq - 1) mma_commit(kv_free);
+          if (!mbar_wait(p_ready, p_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          ++p_waits;
+          if (i == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO and dK += dS^T Q (queries are the contraction, 8 steps of 16)
+#pragma unroll
+          for (int kk = 0; kk < kBM / 16; ++kk) {
+            const uint32_t off = (kk * 16 * 128) >> 4;
+            mma_ts(tmem + C::kTmDV, tmem + C::kTmS + kk * 8, sm0 + dso + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kBM / 16; ++kk) {
+            const uint32_t off = (kk * 16 * 128) >> 4;
+            mma_ts(tmem + C::kTmDK, tmem + C::kTmDP + kk * 8, sm0 + so + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&st_empty[st]);
+          ++ld;
+        }
+        if (!ok) break;
+        mma_commit(acc_done);
+        ++item_ctr;
+      }
+      if (!ok && issued) {
+        mma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else {
+    // elementwise warps: thread = key row of the block = TMEM lane
+    const int row = warp * 32 + lane;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t ld = 0, s_waits = 0, item_ctr = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
+      int bh, ktile, kb, off0, nq;
+      item_info(item, bh, ktile, kb, off0, nq);
+      const int krow = kb * kBM + row;
+      const bool row_valid = krow < g.tau;
+      for (int i = 0; i < nq; ++i) {
+        const int qb = i % p.nqb;
+        const int valid_q = min(kBM, g.tau - qb * kBM);
+        const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
+        bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
+        ++s_waits;
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) { ok = false; break; }
+        tc_fence_after();
+        const float *lse_s = reinterpret_cast<const float *>(stages + st * C::kStage + 2 * C::kTile);
+        const float *dd_s = lse_s + 128;
+#pragma unroll
+        for (int c = 0; c < kBM / 32; ++c) {
+          uint32_t rs[32], rd[32];
+          tmem_ld32(tmem + lane_off + C::kTmS + c * 32, rs);
+          tmem_ld32(tmem + lane_off + C::kTmDP + c * 32, rd);
+          tmem_ld_wait();
+          uint32_t pp[16], pd[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = c * 32 + e;
+            float pr[2], dr[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const bool v = q + h < valid_q;
+              const float pv = ex2_approx(fmaf(__uint_as_float(rs[e + h]), sl2, -lse_s[q + h]));
+              pr[h] = v ? pv : 0.f;
+              dr[h] = v ? pv * (__uint_as_float(rd[e + h]) - dd_s[q + h]) : 0.f;
+            }
+            pp[e / 2] = pack_bf16(pr[0], pr[1]);
+            pd[e / 2] = pack_bf16(dr[0], dr[1]);
+          }
+          tmem_st16(tmem + lane_off + C::kTmS + c * 16, pp);
+          tmem_st16(tmem + lane_off + C::kTmDP + c * 16, pd);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(p_ready, lane);
+        ++ld;
+      }
+      if (!ok) break;
+      // epilogue: dV, scale * dK -> bf16 rows of this key block
+      bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
+      oke = __all_sync(0xffffffffu, oke);
+      if (!oke) { ok = false; break; }
+      tc_fence_after();
+      const long long tok = row_valid ? token_row(g, p.tiled, bh, ktile, krow) : 0;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? C::kTmDK : C::kTmDV;
+        const float mul = which ? p.scale : 1.f;
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(which ? p.dk : p.dv) + tok * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + col + c * 32, r);
+          tmem_ld_wait();
+          if (row_valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
+              w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
+              w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
+              w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
+              dst[c * 4 + v] = w;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      warp_arrive(acc_free, lane);
+      ++item_ctr;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------------- 3. dQ
+template <int D>
+struct DqCfg {
+  static constexpr uint32_t kTile = kBM * D * 2;
+  static constexpr uint32_t kPanel = kBM * 128;
+  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr int kNumBars = 2 * kSlots + 7;
+  static constexpr uint32_t kSmem = (2 + kSlots) * kTile + kNumBars * 8 + 64 + 16 + kMaxCoords * 16 + 1024;
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDQ = 256;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
+                  const BwdParams p) {
+  using C = DqCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *q_s = smem, *do_s = smem + C::kTile, *slots = smem + 2 * C::kTile;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(slots + C::kSlots * C::kTile);
+  uint64_t *full = bars, *empty = bars + C::kSlots;
+  uint64_t *q_full = bars + 2 * C::kSlots, *q_free = q_full + 1, *s_full = q_full + 2, *ds_ready = q_full + 3;
+  uint64_t *acc_done = q_full + 4, *acc_free = q_full + 5, *drain = q_full + 6;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int4 *s_coord = reinterpret_cast<int4 *>((reinterpret_cast<uintptr_t>(tmem_slot) + 64 + 15) & ~uintptr_t(15));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Geometry &g = p.g;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kSlots; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
+    mbar_init(s_full, 1);
+    mbar_init(ds_ready, 4);
+    mbar_init(acc_done, 1);
+    mbar_init(acc_free, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+  const int pieces = kBM / p.piece_rows;
+
+  struct Item {
+    int bh, tile, qb, head, nkeys, nc;
+  };
+  auto item_info = [&](int item) {
+    const int2 wi = p.work_q[item];
+    Item it;
+    it.bh = wi.x, it.tile = wi.y / p.nqb, it.qb = wi.y % p.nqb, it.head = it.bh % g.Hh;
+    it.nkeys = p.kv_count[it.head] * g.tau;
+    it.nc = (it.nkeys + kBM - 1) / kBM;
+    return it;
+  };
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      tma_prefetch_desc(&tmap_do);
+    }
+    uint32_t ld = 0, item_ctr = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
+      const Item it = item_info(item);
+      const int32_t *list = p.kv_list + ((long long)it.head * g.n_tiles + it.tile) * p.kv_stride;
+      const int nbox = it.nc * pieces;
+      const bool staged = nbox <= kMaxCoords;
+      auto kv_coord = [&](int e) -> int4 {
+        const int key = (e / pieces) * kBM + (e % pieces) * p.piece_rows;
+        const bool valid = key < it.nkeys;
+        const int li = key / g.tau;
+        return box_coords(p, it.bh, valid ? __ldg(list + li) : 0, key - li * g.tau, valid);
+      };
+      __syncwarp();
+      if (staged)
+        for (int e = lane; e < nbox; e += 32) s_coord[e] = kv_coord(e);
+      __syncwarp();
+      if (lane == 0) {
+        if (!mbar_wait(q_free, (item_ctr & 1) ^ 1, ctl, kErrBwdWait)) ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(q_full, 2 * C::kTile);
+          for (int pc = 0; pc < pieces; ++pc) {
+            const int off = it.qb * kBM + pc * p.piece_rows;
+            const int4 c = box_coords(p, it.bh, it.tile, off, off < g.tau);
+            load_box<D>(p, &tmap_q, q_s + pc * p.piece_rows * 128, c, q_full);
+            load_box<D>(p, &tmap_do, do_s + pc * p.piece_rows * 128, c, q_full);
+          }
+        }
+        for (int s = 0; s < 2 * it.nc && ok; ++s) {
+          const int chunk = s >> 1, is_v = s & 1;
+          const uint32_t slot = ld % C::kSlots, phase = (ld / C::kSlots) & 1;
+          if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrBwdWait)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[slot], C::kTile);
+          for (int pc = 0; pc < pieces; ++pc) {
+            const int e = chunk * pieces + pc;
+            load_box<D>(p, is_v ? &tmap_v : &tmap_k, slots + slot * C::kTile + pc * p.piece_rows * 128,
+                        staged ? s_coord[e] : kv_coord(e), &full[slot]);
+          }
+          ++ld;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ld = __shfl_sync(0xffffffffu, ld, 0);
+      ++item_ctr;
+    }
+    if (!ok && lane == 0) {
+      const uint32_t first = ld > (uint32_t)C::kSlots ? ld - C::kSlots : 0;
+      for (uint32_t i = first; i < ld; ++i) drain_wait(&full[i % C::kSlots], (i / C::kSlots) & 1);
+      if (item_ctr > 0) drain_wait(q_full, (item_ctr - 1) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(kBM, D, false, true);
+      const uint64_t qd = smem_desc_sw128(smem_u32(q_s), 16, 1024), dod = smem_desc_sw128(smem_u32(do_s), 16, 1024);
+      const uint64_t sk0 = smem_desc_sw128(smem_u32(slots), 16, 1024);         // K-major K / V
+      const uint64_t sm0 = smem_desc_sw128(smem_u32(slots), C::kPanel, 1024);  // MN-major K
+      uint32_t ld = 0, item_ctr = 0, ds_waits = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
+        const Item it = item_info(item);
+        if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
+        tc_fence_after();
+        for (int j = 0; j < it.nc && ok; ++j) {
+          const uint32_t lk = ld + 2 * j, lv = lk + 1;
+          const uint32_t ks = lk % C::kSlots, vs = lv % C::kSlots;
+          if (!mbar_wait(&full[ks], (lk / C::kSlots) & 1, ctl, kErrBwdWait) ||
+              !mbar_wait(&full[vs], (lv / C::kSlots) & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + C::kTmS, qd + off, sk0 + ((ks * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+            mma_ss(tmem + C::kTmDP, dod + off, sk0 + ((vs * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit(s_full);
+          mma_commit(&empty[vs]);
+          if (j == it.nc - 1) mma_commit(q_free);
+          if (!mbar_wait(ds_ready, ds_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          ++ds_waits;
+          if (j == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          tc_fence_after();
+          // dQ += dS K (keys are the contraction)
+#pragma unroll
+          for (int kk = 0; kk < kBM / 16; ++kk)
+            mma_ts(tmem + C::kTmDQ, tmem + C::kTmS + kk * 8, sm0 + ((ks * C::kTile + kk * 16 * 128) >> 4), idesc_dq,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[ks]);
+        }
+        if (!ok) break;
+        ld += 2 * it.nc;
+        mma_commit(acc_done);
+        ++item_ctr;
+      }
+      if (!ok && issued) {
+        mma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else {
+    const int row = warp * 32 + lane;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t s_waits = 0, item_ctr = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
+      const Item it = item_info(item);
+      const int qrow = it.qb * kBM + row;
+      const bool row_valid = qrow < g.tau;
+      const long long lo = it.bh * lse_pitch(g) + (long long)it.tile * g.tau + qrow;
+      const float lse2 = row_valid ? p.lse2_t[lo] : 0.f, dd = row_valid ? p.dd_t[lo] : 0.f;
+      for (int j = 0; j < it.nc; ++j) {
+        bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
+        ++s_waits;
+        okw = __all_sync(0xffffffffu, okw);
+        if (!okw) { ok = false; break; }
+        tc_fence_after();
+        const int kvalid = it.nkeys - j * kBM;
+#pragma unroll
+        for (int c = 0; c < kBM / 32; ++c) {
+          uint32_t rs[32], rd[32];
+          tmem_ld32(tmem + lane_off + C::kTmS + c * 32, rs);
+          tmem_ld32(tmem + lane_off + C::kTmDP + c * 32, rd);
+          tmem_ld_wait();
+          uint32_t pd[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float dr[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const bool v = c * 32 + e + h < kvalid;
+              const float pv = ex2_approx(fmaf(__uint_as_float(rs[e + h]), sl2, -lse2));
+              dr[h] = v ? pv * (__uint_as_float(rd[e + h]) - dd) : 0.f;
+            }
+            pd[e / 2] = pack_bf16(dr[0], dr[1]);
+          }
+          tmem_st16(tmem + lane_off + C::kTmS + c * 16, pd);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(ds_ready, lane);
+      }
+      if (!ok) break;
+      bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
+      oke = __all_sync(0xffffffffu, oke);
+      if (!oke) { ok = false; break; }
+      tc_fence_after();
+      const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, qrow) : 0;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dq) + tok * D);
+      const float mul = p.scale;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + C::kTmDQ + c * 32, r);
+        tmem_ld_wait();
+        if (row_valid) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
+            w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
+            w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
+            w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
+            dst[c * 4 + v] = w;
+          }
+        }
+      }
+      tc_fence_before();
+      warp_arrive(acc_free, lane);
+      ++item_ctr;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const CUtensorMap &tdo, int num_sms, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)DkvCfg<D>::kSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DqCfg<D>::kSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const long long rows = (long long)p.g.B * p.g.Hh * p.g.N;
+  long long pre_blocks = (rows + 7) / 8;
+  if (pre_blocks > (long long)num_sms * 16) pre_blocks = (long long)num_sms * 16;
+  bwd_pre_kernel<D><<<(int)pre_blocks, 256, 0, stream>>>(p);
+  const int g1 = p.n_work_kv < num_sms ? p.n_work_kv : num_sms;
+  if (g1 > 0) bwd_dkdv_kernel<D><<<g1, kThreads, DkvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  const int g2 = p.n_work_q < num_sms ? p.n_work_q : num_sms;
+  if (g2 > 0) bwd_dq_kernel<D><<<g2, kThreads, DqCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                            const CUtensorMap &tmap_v, const CUtensorMap &tmap_do, int num_sms,
+                            cudaStream_t stream) {
+  if (p.g.d == 128) return launch_bwd_d<128>(p, tmap_q, tmap_k, tmap_v, tmap_do, num_sms, stream);
+  if (p.g.d == 64) return launch_bwd_d<64>(p, tmap_q, tmap_k, tmap_v, tmap_do, num_sms, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sta

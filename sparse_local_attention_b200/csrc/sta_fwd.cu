@@ -35,6 +35,7 @@
 
 #include "sm100_ptx.cuh"
 #include "sta_kernels.h"
+#include "sta_common.cuh"
 
 namespace sta {
 namespace {
@@ -44,7 +45,6 @@ constexpr int kBN = 128;  // keys per chunk (MMA N of Q K^T, K of P V)
 constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kMaxCoords = 1024;  // per-item K/V box coordinates staged in shared memory
-constexpr uint64_t kDrainLimitNs = 200ull * 1000 * 1000;  // 0.2 s
 
 template <int D>
 struct FwdCfg {
@@ -63,28 +63,6 @@ struct FwdCfg {
   static_assert(kTmO0 + 2 * D <= kTmCols, "TMEM budget");
 };
 
-__device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > (long long)(2 * kDrainLimitNs)) return false;
-  return true;
-}
-
-// Token index (in the tensor's own order) of row `o` of query tile `tile`.
-__device__ __forceinline__ long long token_row(const Geometry &g, int tiled, int bh, int tile, int o) {
-  if (tiled) return (long long)bh * g.N + (long long)tile * g.tau + o;
-  const int it = tile / (g.GH * g.GW), ih = (tile / g.GW) % g.GH, iw = tile % g.GW;
-  const int a = o / (g.th * g.tw), b = (o / g.tw) % g.th, c = o % g.tw;
-  const int t = it * g.tt + a, h = ih * g.th + b, w = iw * g.tw + c;
-  return (long long)bh * g.N + ((long long)t * g.H + h) * g.W + w;
-}
-
-// Per-warp arrive: every lane has finished its part before lane 0 arrives.
-__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
-  __syncwarp();
-  if (lane == 0) mbar_arrive(bar);
-}
-
 struct ItemInfo {
   int bh, tile, head, qa;  // qa = first query block of the pair
   bool has_b;
@@ -102,35 +80,6 @@ __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
   it.nkeys = p.kv_count[it.head] * p.g.tau;
   it.nc = (it.nkeys + kBN - 1) / kBN;
   return it;
-}
-
-// TMA box coordinates of `piece_rows` consecutive tile-major rows starting at
-// in-tile row `off` of tile `tile` in slice bh; an out-of-range coordinate
-// (zero fill) when !valid.  Tiled maps use (row); raster maps (w, h, t*bh).
-__device__ __forceinline__ int4 box_coords(const FwdParams &p, int bh, int tile, int off, bool valid) {
-  const Geometry &g = p.g;
-  if (p.kv_mode == kKvTiled) return make_int4(valid ? bh * g.N + tile * g.tau + off : p.oob_coord, 0, 0, 0);
-  const int kt = tile / (g.GH * g.GW), kh = (tile / g.GW) % g.GH, kw = tile % g.GW;
-  const int a = off / (g.th * g.tw), b = (off / g.tw) % g.th, c = off % g.tw;
-  return make_int4(kw * g.tw + c, kh * g.th + b, valid ? bh * g.T + kt * g.tt + a : p.oob_coord, 0);
-}
-
-// Issue the TMA box(es) of one piece (all 64-column panels) at `c`.
-template <int D>
-__device__ __forceinline__ void load_box(const FwdParams &p, const CUtensorMap *map, uint8_t *dst, int4 c,
-                                         uint64_t *bar) {
-  using C = FwdCfg<D>;
-  const int boxes = C::kPanels / p.box_panels;
-  for (int pn = 0; pn < boxes; ++pn) {
-    uint8_t *pdst = dst + pn * C::kPanelBytes;
-    if (p.kv_mode == kKvTiled) {
-      if constexpr (D == 128) tma_load_3d(pdst, map, 0, c.x, pn, bar);
-      else tma_load_2d(pdst, map, 0, c.x, bar);
-    } else {
-      if constexpr (D == 128) tma_load_5d(pdst, map, 0, c.x, c.y, c.z, pn, bar);
-      else tma_load_4d(pdst, map, 0, c.x, c.y, c.z, bar);
-    }
-  }
 }
 
 template <int D>

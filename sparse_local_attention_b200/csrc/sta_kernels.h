@@ -57,6 +57,28 @@ struct FwdParams {
   int oob_coord;             // row (tiled) or T*B*Hh (raster) coordinate past the end
 };
 
+struct BwdParams {
+  Geometry g;
+  int tiled;  // token order of every user tensor (q k v o dout lse dq dk dv)
+  int nqb;    // 128-row blocks per tile = ceil(tau / 128)
+  // operand TMA geometry (same meaning as in FwdParams)
+  int kv_mode, piece_rows, box_w, box_h, box_t, box_panels, oob_coord;
+  const void *o, *dout;  // preprocess inputs
+  const float *lse;      // forward LSE (natural log)
+  float *lse2_t, *dd_t;  // tile-major, pitch N + 128 per slice: LSE*log2(e), D = rowsum(dO*O)
+  void *dq, *dk, *dv;    // bf16 outputs
+  const int32_t *kv_list, *kv_count;  // forward lists (dQ kernel)
+  int kv_stride;
+  const int32_t *inv_off, *inv_idx;   // inverse lists, [Hh][n_tiles + 1] absolute offsets (dK/dV kernel)
+  const int2 *work_kv;                // (bh, key tile * nqb + key block), heaviest first
+  int n_work_kv;
+  const int2 *work_q;                 // (bh, query tile * nqb + query block), heaviest first
+  int n_work_q;
+  float scale, scale_log2;
+  int *status;
+  unsigned long long wait_limit_ns;
+};
+
 struct PermuteParams {
   Geometry g;
   const void *src;
@@ -67,5 +89,10 @@ struct PermuteParams {
 cudaError_t launch_forward(const FwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
                            const CUtensorMap &tmap_v, int num_sms, cudaStream_t stream);
 cudaError_t launch_permute(const PermuteParams &p, int num_sms, cudaStream_t stream);
+// Backward: preprocess (D, LSE*log2 e), dK/dV (key-block major) and dQ
+// (query-block major), enqueued in that order on `stream`.
+cudaError_t launch_backward(const BwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
+                            const CUtensorMap &tmap_v, const CUtensorMap &tmap_do, int num_sms,
+                            cudaStream_t stream);
 
 }  // namespace sta
