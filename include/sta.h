@@ -149,6 +149,29 @@ sta_status sta_backward(sta_plan_t plan, const void *q, const void *k, const voi
                         void *dv, void *workspace, size_t workspace_bytes, void *stream,
                         uint32_t flags);
 
+/* sta_backward without a caller workspace.  (No counterpart in the paper: this
+ * is a calling convention of this library.)  Meant for callers that cannot
+ * allocate device memory where they run the backward pass -- for example when
+ * a framework's caching allocator already owns the whole device, or on a path
+ * where the memory footprint must not change once set up -- and so cannot hand
+ * over a workspace.  The temporaries go to a file-scope device array of 32 MiB
+ * inside libsta.so instead; every GPU that loads the library holds that array
+ * until the process exits.  Same arguments, results and flags as sta_backward,
+ * minus the workspace.
+ *   - Fails with STA_ERR_WORKSPACE when the plan's backward workspace
+ *     (sta_plan_workspace_size, bwd_bytes) exceeds 32 MiB.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ *   - All calls share the one array, which keeps the previous call's contents;
+ *     the status word is cleared on each call and the rest is rewritten before
+ *     use.  Calls that overlap on the GPU (other streams, other host threads on
+ *     the same device) race on it: order them. */
+sta_status sta_backward_noalloc(sta_plan_t plan, const void *q, const void *k, const void *v,
+                                const void *o, const float *lse, const void *dout, void *dq,
+                                void *dk, void *dv, void *stream, uint32_t flags);
+
 /* Process-wide limit, in nanoseconds, on every barrier wait inside the
  * kernels launched after this call (default 2 s).  When a wait runs out the
  * kernel stops early, records the error in the workspace status word and

@@ -27,7 +27,7 @@ STA_CALL_CHECK = 0x1
 
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
             "sta_plan_q_tiles", "sta_plan_geometry", "sta_permute", "sta_forward", "sta_backward",
-            "sta_status_string", "sta_set_wait_limit_ns"]
+            "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc"]
 
 
 class StaError(RuntimeError):
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
     L.sta_permute.argtypes = [vp, vp, vp, ctypes.c_int32, vp]
     L.sta_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
     L.sta_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
+    L.sta_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32]
     L.sta_status_string.argtypes = [ctypes.c_int]
     L.sta_status_string.restype = ctypes.c_char_p
     L.sta_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -248,6 +249,25 @@ def sta_backward(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, w
                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream),
                             STA_CALL_CHECK if check else 0)
     _check(st, "sta_backward")
+    return dq, dk, dv
+
+
+def sta_backward_noalloc(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, stream=None,
+                         check: bool = False):
+    """sta_backward with the library's fixed device scratch instead of a
+    workspace (see include/sta.h).  Output tensors may be passed in; if they
+    are not, they are created here by the caller's allocator (torch)."""
+    p = plan.problem
+    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _expect(t, nm, shape, torch.bfloat16)
+    _expect(lse, "lse", shape[:3], torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib().sta_backward_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream), STA_CALL_CHECK if check else 0)
+    _check(st, "sta_backward_noalloc")
     return dq, dk, dv
 
 
