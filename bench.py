@@ -229,7 +229,7 @@ def run_ours(args):
 
     q_h, k_h, v_h = (x.pin_memory() for x in make_inputs(wl, seed=rank))
     q, k, v = (x.cuda() for x in (q_h, k_h, v_h))
-    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=wl.backward))
     o = torch.empty_like(q)
     lse = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32, device="cuda")
     ws = plan.workspace()
@@ -262,6 +262,29 @@ def run_ours(args):
     flops = wl.forward_flops()
     value = flops * world / (ms * 1e-3) / 1e12
     launches_per_step = 1
+
+    # --- backward (fine-tuning workloads): dQ, dK, dV from the same inputs
+    bwd = None
+    if wl.backward:
+        do_h = make_inputs(wl, with_dout=True, seed=rank)[3]
+        dout = do_h.cuda()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = plan.workspace(backward=True)
+        sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws, check=True)
+        for _ in range(args.warmup):
+            sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        bms = max_over_ranks(dist, b0.elapsed_time(b1) / args.steps)
+        bwd = {"ms_per_step": bms, "tflops_useful": wl.backward_flops() * world / (bms * 1e-3) / 1e12,
+               "useful_flop_convention": "2.5 x forward (five GEMM-shaped products)",
+               "kernels_per_step": 3}
+        del dout, dq, dk, dv, bws
 
     # --- end to end through the public API: pinned host in, host out
     o_h = torch.empty_like(q_h).pin_memory()
@@ -338,6 +361,7 @@ def run_ours(args):
             "clocks": clocks,
             "cpu_baseline": cpu,
             "dense_baseline": dense,
+            "backward": bwd,
         }
         print(json.dumps(out), flush=True)
     plan.destroy()
