@@ -63,6 +63,14 @@ typedef enum {
                                       with STA_ERR_INVALID_ARG.  For tooling and
                                       for inspecting lists on machines without
                                       a GPU. */
+#define STA_PROBLEM_CTA_PAIR 0x8u  /* run the forward pass on CTA pairs
+                                      (tcgen05 cta_group::2, M = 256 over two
+                                      SMs, each SM loading half of every K/V
+                                      chunk) where the geometry allows it: head
+                                      dim 128 and a tile volume that is a
+                                      multiple of 128.  Same results; by
+                                      default the one-CTA kernel runs, which is
+                                      faster on every shape measured so far. */
 
 /* flags of sta_forward / sta_backward */
 #define STA_CALL_CHECK 0x1u /* synchronize `stream` after the launch and report

@@ -34,6 +34,8 @@ struct sta_plan_s {
   int npairs = 1;
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
+  bool pair = false;  // forward runs on CTA pairs (sta_fwd_pair.cu)
+  int kh_box[3] = {0, 0, 0}, vh_box[3] = {0, 0, 0};  // raster boxes of 64 and 128 rows
   bool host_only = false;
   bool tiled = false;
   float scale = 0.f;
@@ -105,15 +107,16 @@ EncodeTiledFn encode_fn() {
 // when the chunk is a single piece and d = 128; otherwise one panel per box.
 int box_panels(const sta_plan_s *pl) { return (pl->g.d == 128 && pl->piece_rows == 128) ? 2 : 1; }
 
-// Tile-major buffer [rows][d] bf16: (64, rows[, 2 panels]), box (64, piece_rows[, panels]).
-bool make_map_tiled(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+// Tile-major buffer [rows][d] bf16 viewed as (64, rows[, 2 panels]); a box is
+// `box_rows` rows by `panels` 64-column panels.
+bool make_map_tiled_box(CUtensorMap *m, const void *base, const sta_plan_s *pl, int box_rows, int panels) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const Geometry &g = pl->g;
   const cuuint64_t rows = (cuuint64_t)g.B * g.Hh * g.N;
   cuuint64_t dims[3] = {64, rows, 2};
   cuuint64_t strides[2] = {(cuuint64_t)g.d * 2, 128};
-  cuuint32_t box[3] = {64, (cuuint32_t)pl->piece_rows, (cuuint32_t)box_panels(pl)};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)panels};
   cuuint32_t estr[3] = {1, 1, 1};
   const cuuint32_t rank = g.d == 128 ? 3 : 2;
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
@@ -121,23 +124,31 @@ bool make_map_tiled(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Raster tensor: (64, W, H, T*B*Hh[, 2 panels]); one box = one piece of a tile
-// (whole w-runs and h-planes), so K/V tiles are gathered straight from the
-// raster layout with no permutation pass.
-bool make_map_raster(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+// Raster tensor viewed as (64, W, H, T*B*Hh[, 2 panels]); a box is a run of
+// whole w-lines / h-planes of one tile (bw x bh x bt tokens) by `panels`
+// 64-column panels, so tiles are gathered straight from the raster layout.
+bool make_map_raster_box(CUtensorMap *m, const void *base, const sta_plan_s *pl, int bw, int bh, int bt,
+                         int panels) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const Geometry &g = pl->g;
   const cuuint64_t row = (cuuint64_t)g.d * 2;
   cuuint64_t dims[5] = {64, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T * g.B * g.Hh, 2};
   cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, 128};
-  cuuint32_t box[5] = {64, (cuuint32_t)pl->box_w, (cuuint32_t)pl->box_h, (cuuint32_t)pl->box_t,
-                       (cuuint32_t)box_panels(pl)};
+  cuuint32_t box[5] = {64, (cuuint32_t)bw, (cuuint32_t)bh, (cuuint32_t)bt, (cuuint32_t)panels};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const cuuint32_t rank = g.d == 128 ? 5 : 4;
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_tiled(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+  return make_map_tiled_box(m, base, pl, pl->piece_rows, box_panels(pl));
+}
+
+bool make_map_raster(CUtensorMap *m, const void *base, const sta_plan_s *pl) {
+  return make_map_raster_box(m, base, pl, pl->box_w, pl->box_h, pl->box_t, box_panels(pl));
 }
 
 void free_device(sta_plan_s *pl) {
@@ -224,7 +235,7 @@ void sta_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
 
 sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
   if (!prob || !out || !prob->window) return STA_ERR_INVALID_ARG;
-  const uint32_t known = STA_PROBLEM_BACKWARD | STA_PROBLEM_TILED | STA_PROBLEM_HOST_ONLY;
+  const uint32_t known = STA_PROBLEM_BACKWARD | STA_PROBLEM_TILED | STA_PROBLEM_HOST_ONLY | STA_PROBLEM_CTA_PAIR;
   if (prob->flags & ~known) return STA_ERR_INVALID_ARG;
   if (prob->batch < 1 || prob->heads < 1 || prob->T < 1 || prob->H < 1 || prob->W < 1 || prob->tile_t < 1 ||
       prob->tile_h < 1 || prob->tile_w < 1)
@@ -308,10 +319,14 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       }
     }
 
-    // --- forward work items: pairs of 128-row query blocks of one tile.
-    //     Heaviest heads first (longest-processing-time order for the
-    //     persistent grid); within a head, tile by tile, so consecutive items
-    //     share most of their key tiles in L2.
+    // --- forward work items: pairs of 128-row query blocks of one tile (the
+    //     last item of a tile with an odd number of blocks has one block).
+    //     The persistent grid takes items round-robin, so they are ordered by
+    //     cost, largest first (query blocks x key tiles: a longest-processing-
+    //     time order); within a cost, head by head and tile by tile, so
+    //     consecutive items share most of their key tiles in L2.  Ordering by
+    //     cost also keeps the two kinds of item from lining up with the grid
+    //     stride (every CTA would otherwise get only one kind).
     std::vector<int> heads(g.Hh);
     std::iota(heads.begin(), heads.end(), 0);
     std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
@@ -320,6 +335,14 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       for (int b = 0; b < g.B; ++b)
         for (int t = 0; t < g.n_tiles; ++t)
           for (int pr = 0; pr < pl->npairs; ++pr) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
+    {
+      const int nqb = (g.tau + 127) / 128;
+      auto cost = [&](const int2 &w) {
+        const int pr = w.y % pl->npairs;
+        return (long long)std::min(2, nqb - 2 * pr) * pl->count[w.x % g.Hh];
+      };
+      std::stable_sort(pl->work.begin(), pl->work.end(), [&](const int2 &a, const int2 &b) { return cost(a) > cost(b); });
+    }
 
     if (prob->flags & STA_PROBLEM_BACKWARD) {
       const int nqb = (g.tau + 127) / 128;
@@ -354,6 +377,17 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     pl->kv_mode = sta::kKvRaster;
   } else {
     pl->kv_mode = sta::kKvTiled;  // permute K and V into the workspace first
+  }
+
+  // CTA-pair forward (on request): head dim 128, whole 128-row chunks inside a
+  // tile, and (for raster inputs read in place) 64- and 128-row runs that are boxes.
+  if ((prob->flags & STA_PROBLEM_CTA_PAIR) && g.d == 128 && g.tau % 128 == 0) {
+    if (pl->kv_mode == sta::kKvTiled) {
+      pl->pair = true;
+    } else {
+      pl->pair = raster_box(g, 64, &pl->kh_box[0], &pl->kh_box[1], &pl->kh_box[2]) &&
+                 raster_box(g, 128, &pl->vh_box[0], &pl->vh_box[1], &pl->vh_box[2]);
+    }
   }
 
   if (!pl->host_only) {
@@ -504,7 +538,16 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
 
   if (flags & STA_CALL_CHECK)
     if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;
-  if (sta::launch_forward(fp, mq, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+  if (pl->pair) {
+    CUtensorMap mkh, mvh;
+    const bool okp = raster5d ? (make_map_raster_box(&mkh, kbase, pl, pl->kh_box[0], pl->kh_box[1], pl->kh_box[2], 2) &&
+                                 make_map_raster_box(&mvh, vbase, pl, pl->vh_box[0], pl->vh_box[1], pl->vh_box[2], 1))
+                              : (make_map_tiled_box(&mkh, kbase, pl, 64, 2) && make_map_tiled_box(&mvh, vbase, pl, 128, 1));
+    if (!okp) return STA_ERR_CUDA;
+    if (sta::launch_forward_pair(fp, mkh, mvh, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+  } else {
+    if (sta::launch_forward(fp, mq, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
+  }
   return finish_call(pl, workspace, stream, flags);
 }
 

@@ -10,7 +10,11 @@
 //     query blocks (A, B) of the same query tile -- both attend to the same
 //     key tiles, so every K/V chunk brought into shared memory serves 256
 //     query rows.  When a tile has an odd number of blocks the last item has
-//     block A only.  Items are ordered heaviest head first.
+//     one block; its key chunks are then divided between the two warpgroups
+//     (the first half to A, the rest to B, both reading the same Q) and the
+//     epilogue merges the two partial softmax states, so a lone block still
+//     keeps two MMA/softmax chains in flight.  Items are ordered heaviest head
+//     first.
 //   * warp 8: TMA producer.  Loads Q_A, Q_B (shared memory, 128-byte swizzle)
 //     and streams K and V chunks of 128 keys into a ring of stages, gathering
 //     them tile by tile from the KV-tile list.  At the start of an item the
@@ -56,7 +60,7 @@ struct FwdCfg {
   static constexpr uint32_t kTmCols = 512;
   // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain
   static constexpr int kNumBars = 2 * kSlots + 11;
-  static constexpr uint32_t kMiscBytes = 64;  // tmem address, abort flag
+  static constexpr uint32_t kMiscBytes = 64 + 4 * 128 * 4;  // tmem address, abort flag, m/l exchange
   static constexpr uint32_t kListBytes = kMaxCoords * 16;
   static constexpr uint32_t kSmemBytes =
       (2 + kSlots) * kTileBytes + kNumBars * 8 + kMiscBytes + 16 + kListBytes + 1024;
@@ -65,8 +69,12 @@ struct FwdCfg {
 
 struct ItemInfo {
   int bh, tile, head, qa;  // qa = first query block of the pair
-  bool has_b;
+  bool has_b;              // a second query block (qa + 1) shares the K/V chunks
+  bool split;              // one query block, its chunks divided between the two warpgroups
   int nkeys, nc;
+  int n0, n1, c1;          // chunks of warpgroup 0: 0 .. n0 - 1; of warpgroup 1: c1 .. c1 + n1 - 1
+  __device__ __forceinline__ int n(int x) const { return x ? n1 : n0; }
+  __device__ __forceinline__ int c0(int x) const { return x ? c1 : 0; }
 };
 
 __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
@@ -79,6 +87,10 @@ __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
   it.has_b = (it.qa + 1) * kBM < p.g.tau;
   it.nkeys = p.kv_count[it.head] * p.g.tau;
   it.nc = (it.nkeys + kBN - 1) / kBN;
+  it.split = !it.has_b && it.nc > 1;
+  it.n0 = it.split ? (it.nc + 1) / 2 : it.nc;
+  it.n1 = it.split ? it.nc - it.n0 : (it.has_b ? it.nc : 0);
+  it.c1 = it.split ? it.n0 : 0;
   return it;
 }
 
@@ -103,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain = o_free + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *ml_xchg = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(tmem_slot) + 64);  // [m0 m1 l0 l1][128]
   int4 *s_coord =  // 16-byte aligned for the int4 accesses
       reinterpret_cast<int4 *>((reinterpret_cast<uintptr_t>(tmem_slot) + C::kMiscBytes + 15) & ~uintptr_t(15));
 
@@ -173,11 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                           box_coords(p, it.bh, it.tile, off, off < g.tau), q_full);
             }
         }
-        // K and V chunks in the order the MMA first uses them: K0 V0 K1 V1 ...
-        for (int s = 0; s < 2 * it.nc && ok; ++s) {
-          const int chunk = s >> 1, is_v = s & 1;
+        // K and V chunks in the order the MMA uses them.  Shared chunks (one
+        // or two blocks): K0 V0 K1 V1 ...  Split item: K_A(0) K_B(0), then per
+        // step j: V_A(j) K_A(j+1) V_B(j) K_B(j+1), where warpgroup x's step j
+        // is chunk c0(x) + j.
+        auto emit = [&](int chunk, int is_v) -> bool {
           const uint32_t slot = ld % C::kSlots, phase = (ld / C::kSlots) & 1;
-          if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrWaitProducer)) { ok = false; break; }
+          if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrWaitProducer)) return false;
           mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
           uint8_t *dst = slots + slot * C::kTileBytes;
           for (int pc = 0; pc < pieces; ++pc) {
@@ -186,7 +201,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         staged ? s_coord[e] : kv_coord(e), &full[slot]);
           }
           ++ld;
-        }
+          return true;
+        };
+        const int nxk = it.split ? 2 : 1;  // K/V streams
+        for (int x = 0; x < nxk && ok; ++x) ok = emit(it.c0(x), 0);
+        for (int j = 0; j < it.n(0) && ok; ++j)
+          for (int x = 0; x < nxk && ok; ++x) {
+            if (j >= it.n(x)) continue;
+            ok = emit(it.c0(x) + j, 1);
+            if (ok && j + 1 < it.n(x)) ok = emit(it.c0(x) + j + 1, 0);
+          }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       ld = __shfl_sync(0xffffffffu, ld, 0);
@@ -214,9 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qdesc0 = smem_desc_sw128(q_addr, 16, 1024);
       const uint64_t kdesc0 = smem_desc_sw128(slots_addr, 16, 1024);
       const uint64_t vdesc0 = smem_desc_sw128(slots_addr, C::kPanelBytes, 1024);
-      // S_X = Q_X K^T for the K chunk in ring slot `slot`.
-      auto mma_s = [&](int x, uint32_t slot) {
-        const uint64_t qd = qdesc0 + ((x * C::kTileBytes) >> 4), kd = kdesc0 + ((slot * C::kTileBytes) >> 4);
+      // S_X = Q_qx K^T for the K chunk in ring slot `slot` (qx = x, or 0 in a split item).
+      auto mma_s = [&](int x, int qx, uint32_t slot) {
+        const uint64_t qd = qdesc0 + ((qx * C::kTileBytes) >> 4), kd = kdesc0 + ((slot * C::kTileBytes) >> 4);
         const uint32_t d_tm = tmem + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -243,42 +267,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
         const ItemInfo it = decode_item(p, item);
-        const int nx = it.has_b ? 2 : 1;
+        const int nx = (it.has_b || it.split) ? 2 : 1;
+        const bool shared_kv = !it.split;  // block B reads block A's ring slots
         if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
         tc_fence_after();
-        // chunk 0: S_A(0) [, S_B(0)]
-        const uint32_t k0 = ld;
-        if (!wait_slot(k0)) { ok = false; break; }
-        for (int x = 0; x < nx; ++x) mma_s(x, k0 % C::kSlots);
-        issued = true;
-        mma_commit(&empty[k0 % C::kSlots]);
-        if (it.nc == 1) mma_commit(q_free);
-        for (int j = 0; j < it.nc && ok; ++j) {
-          const uint32_t vj = k0 + 2 * j + 1, kn = k0 + 2 * j + 2;  // V_j, K_{j+1} load indices
+        uint32_t l = ld, kslot = 0, vslot = 0;
+        int s_left = it.nc;  // S groups still to issue (one per chunk)
+        // The ring slot for warpgroup x's next K or V: shared chunks reuse A's.
+        auto take = [&](int x, uint32_t &slot) -> bool {
+          if (x == 1 && shared_kv) return true;
+          if (!wait_slot(l)) return false;
+          slot = l++;
+          return true;
+        };
+        auto release = [&](int x, uint32_t slot) {
+          if (!shared_kv || x == nx - 1) mma_commit(&empty[slot % C::kSlots]);
+        };
+        auto s_group_done = [&](int x) {
+          if (shared_kv && x != nx - 1) return;
+          if (--s_left == 0) mma_commit(q_free);  // Q is no longer read
+        };
+        // first chunk of each warpgroup
+        for (int x = 0; x < nx && ok; ++x) {
+          if (!take(x, kslot)) { ok = false; break; }
+          mma_s(x, it.split ? 0 : x, kslot % C::kSlots);
+          issued = true;
+          release(x, kslot);
+          s_group_done(x);
+        }
+        for (int j = 0; j < it.n(0) && ok; ++j) {
           for (int x = 0; x < nx; ++x) {
+            if (j >= it.n(x)) continue;
             if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
             ++p_waits[x];
             tc_fence_after();
             if (j == 0 && x_items[x] > 0) {
-              // the previous item of this block has read O_X in its epilogue
+              // the previous item of this warpgroup has read O_X in its epilogue
               if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
               ++o_waits[x];
               tc_fence_after();
             }
-            if (x == 0 && !wait_slot(vj)) { ok = false; break; }
-            mma_pv(x, vj % C::kSlots, j == 0);
-            if (x == nx - 1) mma_commit(&empty[vj % C::kSlots]);
-            if (j + 1 < it.nc) {
-              if (x == 0 && !wait_slot(kn)) { ok = false; break; }
-              mma_s(x, kn % C::kSlots);
-              if (x == nx - 1) {
-                mma_commit(&empty[kn % C::kSlots]);
-                if (j + 2 == it.nc) mma_commit(q_free);
-              }
+            if (!take(x, vslot)) { ok = false; break; }
+            mma_pv(x, vslot % C::kSlots, j == 0);
+            release(x, vslot);
+            if (j + 1 < it.n(x)) {
+              if (!take(x, kslot)) { ok = false; break; }
+              mma_s(x, it.split ? 0 : x, kslot % C::kSlots);
+              release(x, kslot);
+              s_group_done(x);
             }
           }
         }
-        ld = k0 + 2 * it.nc;
+        ld = l;
         for (int x = 0; x < nx; ++x) ++x_items[x];
         ++item_ctr;
       }
@@ -290,6 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax: warpgroup x owns block x
+    // (in a split item: the chunks c0(x) .. c0(x) + n(x) - 1 of block A's keys)
     const int x = warp >> 2;
     const int quad = warp & 3;         // TMEM lane quadrant
     const int row = quad * 32 + lane;  // query row of the block = TMEM lane
@@ -297,16 +338,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_col = 128 * x, o_col = C::kTmO0 + x * D;
     const float sl2 = p.scale_log2;
     uint32_t s_waits = 0, pv_waits = 0;
+    // After a failed wait the warpgroup keeps walking the items without
+    // touching barriers or TMEM, so that both warpgroups still meet at the
+    // named barriers of split items.
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
+    for (int item = blockIdx.x; item < p.n_work; item += gridDim.x) {
       const ItemInfo it = decode_item(p, item);
-      if (x == 1 && !it.has_b) continue;
-      const int o_in_tile = (it.qa + x) * kBM + row;
+      if (it.n(x) == 0) continue;
+      const int o_in_tile = (it.qa + (it.split ? 0 : x)) * kBM + row;
       const bool row_valid = o_in_tile < g.tau;
       const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, o_in_tile) : 0;
 
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.nc; ++j) {
+      for (int j = 0; j < it.n(x) && ok; ++j) {
         bool okw = mbar_wait(&s_full[x], s_waits & 1, ctl, kErrWaitSoftmax);
         ++s_waits;
         if (okw && j > 0) {
@@ -334,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             s[96 + i] = __uint_as_float(r3[i]);
           }
         }
-        const int kvalid = it.nkeys - j * kBN;
+        const int kvalid = it.nkeys - (it.c0(x) + j) * kBN;
         if (kvalid < kBN) {
 #pragma unroll
           for (int i = 0; i < kBN; ++i)
@@ -387,13 +431,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         warp_arrive(&p_ready[x], lane);
       }
-      if (!ok) break;
 
       // epilogue: O_X / l -> bf16 row, LSE
-      bool oke = mbar_wait(&pv_done[x], pv_waits & 1, ctl, kErrWaitEpilogue);
-      ++pv_waits;
-      oke = __all_sync(0xffffffffu, oke);
-      if (!oke) { ok = false; break; }
+      bool oke = false;
+      if (ok) {
+        oke = mbar_wait(&pv_done[x], pv_waits & 1, ctl, kErrWaitEpilogue);
+        ++pv_waits;
+        oke = __all_sync(0xffffffffu, oke);
+      }
+      if (it.split) {
+        // Merge the two partial states of the row (m_x, l_x, O_x); warpgroup x
+        // writes output columns [x D / 2, (x + 1) D / 2).
+        ml_xchg[x * 128 + row] = m;
+        ml_xchg[(2 + x) * 128 + row] = l;
+        const bool both = named_bar_and(1, 256, oke);
+        ok = ok && both;
+        if (both) {
+          tc_fence_after();
+          const float m0 = ml_xchg[row], m1 = ml_xchg[128 + row];
+          const float mf = fmaxf(m0, m1);
+          const float a0 = ex2_approx(m0 - mf), a1 = ex2_approx(m1 - mf);
+          const float lf = ml_xchg[256 + row] * a0 + ml_xchg[384 + row] * a1;
+          const float inv_l = 1.f / lf;
+          const float f0 = a0 * inv_l, f1 = a1 * inv_l;
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + tok * D + x * (D / 2));
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tmem + lane_off + C::kTmO0 + x * (D / 2) + c * 32, r0);
+            tmem_ld32(tmem + lane_off + C::kTmO0 + D + x * (D / 2) + c * 32, r1);
+            tmem_ld_wait();
+            if (row_valid) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  o[e] = __uint_as_float(r0[8 * v + e]) * f0 + __uint_as_float(r1[8 * v + e]) * f1;
+                uint4 w;
+                w.x = pack_bf16(o[0], o[1]);
+                w.y = pack_bf16(o[2], o[3]);
+                w.z = pack_bf16(o[4], o[5]);
+                w.w = pack_bf16(o[6], o[7]);
+                dst[c * 4 + v] = w;
+              }
+            }
+          }
+          if (x == 0 && row_valid && p.lse) p.lse[tok] = (mf + __log2f(lf)) * 0.69314718055994530942f;
+          tc_fence_before();
+        }
+        // both warpgroups are done with O_A, O_B and the exchange area
+        named_bar_sync(2, 256);
+        if (both) warp_arrive(&o_free[x], lane);
+        continue;
+      }
+      if (!oke) {
+        ok = false;
+        continue;
+      }
       tc_fence_after();
       const float inv_l = 1.f / l;
       uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + tok * D);

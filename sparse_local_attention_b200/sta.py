@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_SHAPE", 3: "S
 STA_PROBLEM_BACKWARD = 0x1
 STA_PROBLEM_TILED = 0x2
 STA_PROBLEM_HOST_ONLY = 0x4
+STA_PROBLEM_CTA_PAIR = 0x8
 STA_CALL_CHECK = 0x1
 
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
@@ -116,20 +117,21 @@ class Problem:
     backward: bool = False
     tiled: bool = False
     host_only: bool = False
+    cta_pair: bool = False
 
     def _c(self):
         flat = [int(x) for w in self.windows for x in w]
         arr = (ctypes.c_int32 * max(1, len(flat)))(*flat)
         flags = ((STA_PROBLEM_BACKWARD if self.backward else 0) | (STA_PROBLEM_TILED if self.tiled else 0)
-                 | (STA_PROBLEM_HOST_ONLY if self.host_only else 0))
+                 | (STA_PROBLEM_HOST_ONLY if self.host_only else 0) | (STA_PROBLEM_CTA_PAIR if self.cta_pair else 0))
         p = _Problem(self.batch, self.heads, self.head_dim, self.T, self.H, self.W, *self.tile,
                      ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), float(self.scale), flags)
         return p, arr
 
     @staticmethod
-    def from_workload(wl, backward=None, tiled=False, host_only=False, scale=0.0) -> "Problem":
+    def from_workload(wl, backward=None, tiled=False, host_only=False, scale=0.0, cta_pair=False) -> "Problem":
         return Problem(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows), scale,
-                       bool(wl.backward if backward is None else backward), tiled, host_only)
+                       bool(wl.backward if backward is None else backward), tiled, host_only, cta_pair)
 
 
 class Plan:

@@ -24,8 +24,8 @@ def geom_of(wl: Workload) -> Geometry:
     return Geometry(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows))
 
 
-def run_gpu(wl: Workload, q, k, v, tiled=False):
-    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, tiled=tiled))
+def run_gpu(wl: Workload, q, k, v, tiled=False, cta_pair=False):
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, tiled=tiled, cta_pair=cta_pair))
     qd, kd, vd = (x.cuda() for x in (q, k, v))
     o, lse = sta.sta_forward(plan, qd, kd, vd, check=True)
     torch.cuda.synchronize()
@@ -73,6 +73,11 @@ SMALL = {
     "d128_permute_fallback": Workload("e", 1, 2, 128, 4, 12, 8, (2, 6, 4), ((3, 1, 2), (2, 2, 2))),
     "d64_single_tile_grid": Workload("f", 2, 1, 64, 2, 8, 8, (2, 8, 8), ((3, 3, 3),)),
     "d128_tau8_tiny_tiles": Workload("g", 1, 2, 128, 4, 4, 8, (1, 2, 4), ((3, 3, 3), (2, 1, 2))),
+    # tile volumes that are multiples of 128 (also run on CTA pairs below)
+    "d128_pair_tau128_one_block": Workload("h", 1, 2, 128, 4, 16, 16, (2, 8, 8), ((3, 3, 3), (1, 2, 2))),
+    "d128_pair_tau256": Workload("i", 2, 1, 128, 8, 16, 24, (4, 8, 8), ((2, 3, 3),)),
+    "d128_pair_tau384_odd_blocks": Workload("j", 1, 2, 128, 12, 16, 16, (6, 8, 8), ((3, 3, 3), (1, 1, 1))),
+    "d128_pair_tau256_big_window": Workload("k", 1, 1, 128, 8, 24, 24, (4, 8, 8), ((5, 5, 5),)),
 }
 
 
@@ -85,12 +90,33 @@ def test_forward_small_all_rows(name):
     compare_rows(wl, o, lse, q, k, v, rows)
 
 
-def test_forward_tiled_layout_matches_raster():
-    wl = SMALL["d128_tau48_boxes_of_16"]
+PAIR_CASES = [n for n in SMALL if n.startswith("d128_pair")]
+
+
+@pytest.mark.parametrize("name", PAIR_CASES)
+def test_forward_cta_pair_all_rows(name):
+    """The CTA-pair kernel (STA_PROBLEM_CTA_PAIR) against the oracle."""
+    wl = SMALL[name]
+    q, k, v = make_inputs(wl, seed=1)
+    o, lse, _ = run_gpu(wl, q, k, v, cta_pair=True)
+    compare_rows(wl, o, lse, q, k, v, np.arange(wl.B * wl.Hh * wl.N))
+
+
+def test_forward_cta_pair_dit720p_sampled():
+    wl = WORKLOADS["dit720p"]
+    q, k, v = make_inputs(wl)
+    o, lse, _ = run_gpu(wl, q, k, v, cta_pair=True)
+    compare_rows(wl, o, lse, q, k, v, sampled_rows(wl, 32, 6))
+
+
+@pytest.mark.parametrize("name,cta_pair", [("d128_tau48_boxes_of_16", False), ("d128_pair_tau384_odd_blocks", False),
+                                           ("d128_pair_tau384_odd_blocks", True)])
+def test_forward_tiled_layout_matches_raster(name, cta_pair):
+    wl = SMALL[name]
     q, k, v = make_inputs(wl, seed=2)
-    o, lse, plan = run_gpu(wl, q, k, v)
+    o, lse, plan = run_gpu(wl, q, k, v, cta_pair=cta_pair)
     qt, kt, vt = (sta.sta_permute(plan, x.cuda()) for x in (q, k, v))
-    plan_t = sta.sta_plan_create(sta.Problem.from_workload(wl, tiled=True))
+    plan_t = sta.sta_plan_create(sta.Problem.from_workload(wl, tiled=True, cta_pair=cta_pair))
     o_t, lse_t = sta.sta_forward(plan_t, qt, kt, vt, check=True)
     o_back = sta.sta_permute(plan, o_t, inverse=True)
     torch.cuda.synchronize()
