@@ -261,7 +261,7 @@ def run_ours(args):
     ms = max_over_ranks(dist, ms_rank)
     flops = wl.forward_flops()
     value = flops * world / (ms * 1e-3) / 1e12
-    launches_per_step = 1
+    launches_per_step = plan.forward_launches  # kernels one sta_forward call enqueues
 
     # --- backward (fine-tuning workloads): dQ, dK, dV from the same inputs
     bwd = None
@@ -283,7 +283,7 @@ def run_ours(args):
         bms = max_over_ranks(dist, b0.elapsed_time(b1) / args.steps)
         bwd = {"ms_per_step": bms, "tflops_useful": wl.backward_flops() * world / (bms * 1e-3) / 1e12,
                "useful_flop_convention": "2.5 x forward (five GEMM-shaped products)",
-               "kernels_per_step": 3}
+               "kernels_per_step": plan.backward_launches}
         del dout, dq, dk, dv, bws
 
     # --- end to end through the public API: pinned host in, host out

@@ -126,6 +126,14 @@ sta_status sta_plan_q_tiles(sta_plan_t plan, int32_t head, int32_t *offsets, int
 /* Number of tiles of the plan's grid and tokens per tile. */
 sta_status sta_plan_geometry(sta_plan_t plan, int32_t *n_tiles, int32_t *tile_volume);
 
+/* Number of kernels one sta_forward / sta_backward call of this plan enqueues
+ * on its stream (the status-word memset of STA_CALL_CHECK is not counted;
+ * `backward` is 0 for a plan built without STA_PROBLEM_BACKWARD).  For sizing
+ * CUDA-graph captures and for launch accounting.  Either pointer may be NULL;
+ * host-only plans report what a device plan of the same problem launches.
+ * This call has no counterpart in the paper. */
+sta_status sta_plan_launches(sta_plan_t plan, int32_t *forward, int32_t *backward);
+
 /* Token permutation between raster and tile-major order for a bf16 tensor
  * [batch][heads][N][head_dim] of the plan's shape:
  *   inverse == 0: dst[tile-major position of token n] = src[n]   (raster -> tiles)

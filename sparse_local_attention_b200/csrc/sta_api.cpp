@@ -32,6 +32,7 @@ struct sta_plan_s {
   std::vector<int2> work_kv;     // backward dK/dV items (bh, key tile * nqb + key block)
   std::vector<int2> work_q;      // backward dQ items (bh, query tile * nqb + query block)
   int npairs = 1;
+  int n_work_lone = 0;  // forward items with one query block, at the end of `work`
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
   bool pair = false;  // forward runs on CTA pairs (sta_fwd_pair.cu)
@@ -324,9 +325,10 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     //     The persistent grid takes items round-robin, so they are ordered by
     //     cost, largest first (query blocks x key tiles: a longest-processing-
     //     time order); within a cost, head by head and tile by tile, so
-    //     consecutive items share most of their key tiles in L2.  Ordering by
-    //     cost also keeps the two kinds of item from lining up with the grid
-    //     stride (every CTA would otherwise get only one kind).
+    //     consecutive items share most of their key tiles in L2.  The lone
+    //     blocks then move to the end: the one-CTA forward runs them as a
+    //     launch of their own (a grid stride over mixed kinds would hand some
+    //     CTAs only two-block items and others only lone blocks).
     std::vector<int> heads(g.Hh);
     std::iota(heads.begin(), heads.end(), 0);
     std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
@@ -342,6 +344,10 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
         return (long long)std::min(2, nqb - 2 * pr) * pl->count[w.x % g.Hh];
       };
       std::stable_sort(pl->work.begin(), pl->work.end(), [&](const int2 &a, const int2 &b) { return cost(a) > cost(b); });
+      // items with a lone query block last (the one-CTA forward launches them separately)
+      auto lone = [&](const int2 &w) { return 2 * (w.y % pl->npairs) + 1 == nqb; };
+      auto mid = std::stable_partition(pl->work.begin(), pl->work.end(), [&](const int2 &w) { return !lone(w); });
+      pl->n_work_lone = (int)(pl->work.end() - mid);
     }
 
     if (prob->flags & STA_PROBLEM_BACKWARD) {
@@ -440,6 +446,28 @@ sta_status sta_plan_geometry(sta_plan_t pl, int32_t *n_tiles, int32_t *tile_volu
   return STA_OK;
 }
 
+sta_status sta_plan_launches(sta_plan_t pl, int32_t *forward, int32_t *backward) {
+  if (!pl) return STA_ERR_INVALID_ARG;
+  const int n_work = (int)pl->work.size();
+  const bool gather = !pl->tiled && pl->kv_mode != sta::kKvRaster;  // permute Q, K, V (and dO) first
+  if (forward) {
+    int f = gather ? 3 : 0;
+    if (pl->pair) f += n_work > 0 ? 1 : 0;
+    else f += (n_work - pl->n_work_lone > 0 ? 1 : 0) + (pl->n_work_lone > 0 ? 1 : 0);
+    *forward = f;
+  }
+  if (backward) {
+    int b = 0;
+    if (!pl->inv_off.empty()) {
+      b = (gather ? 4 : 0) + 1;  // D / LSE preprocess
+      b += pl->work_kv.empty() ? 0 : 1;
+      b += pl->work_q.empty() ? 0 : 1;
+    }
+    *backward = b;
+  }
+  return STA_OK;
+}
+
 sta_status sta_plan_kv_tiles(sta_plan_t pl, int32_t head, int32_t *out, size_t cap, size_t *n) {
   if (!pl || !n || head < 0 || head >= pl->g.Hh) return STA_ERR_INVALID_ARG;
   const int per = pl->count[head];
@@ -526,7 +554,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   fp.tiled = pl->tiled ? 1 : 0;
   fp.npairs = pl->npairs;
   fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
-  fp.work = pl->d_work, fp.n_work = (int)pl->work.size();
+  fp.work = pl->d_work, fp.n_work = (int)pl->work.size(), fp.n_work_lone = pl->n_work_lone;
   fp.scale_log2 = pl->scale * 1.4426950408889634f;
   fp.status = status;
   fp.wait_limit_ns = g_wait_limit_ns;

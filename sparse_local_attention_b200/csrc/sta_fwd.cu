@@ -13,8 +13,9 @@
 //     one block; its key chunks are then divided between the two warpgroups
 //     (the first half to A, the rest to B, both reading the same Q) and the
 //     epilogue merges the two partial softmax states, so a lone block still
-//     keeps two MMA/softmax chains in flight.  Items are ordered heaviest head
-//     first.
+//     keeps two MMA/softmax chains in flight.  The two kinds of item run as
+//     two launches of two instantiations (kMode 0 / 1), each over its part of
+//     the work list, heaviest items first.
 //   * warp 8: TMA producer.  Loads Q_A, Q_B (shared memory, 128-byte swizzle)
 //     and streams K and V chunks of 128 keys into a ring of stages, gathering
 //     them tile by tile from the KV-tile list.  At the start of an item the
@@ -77,6 +78,11 @@ struct ItemInfo {
   __device__ __forceinline__ int c0(int x) const { return x ? c1 : 0; }
 };
 
+// kMode 0: items of one or two query blocks whose chunks are shared; kMode 1:
+// lone query blocks, their chunks split between the warpgroups when there are
+// at least two.  The host launches one kernel per kind over its part of the
+// work list, so that each instantiation carries only the code it runs.
+template <int kMode>
 __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
   const int2 wi = p.work[item];
   ItemInfo it;
@@ -84,17 +90,17 @@ __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
   it.tile = wi.y / p.npairs;
   it.qa = 2 * (wi.y % p.npairs);
   it.head = it.bh % p.g.Hh;
-  it.has_b = (it.qa + 1) * kBM < p.g.tau;
+  it.has_b = kMode == 0 && (it.qa + 1) * kBM < p.g.tau;
   it.nkeys = p.kv_count[it.head] * p.g.tau;
   it.nc = (it.nkeys + kBN - 1) / kBN;
-  it.split = !it.has_b && it.nc > 1;
+  it.split = kMode == 1 && it.nc > 1;
   it.n0 = it.split ? (it.nc + 1) / 2 : it.nc;
   it.n1 = it.split ? it.nc - it.n0 : (it.has_b ? it.nc : 0);
   it.c1 = it.split ? it.n0 : 0;
   return it;
 }
 
-template <int D>
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
@@ -160,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const int pieces = kBN / p.piece_rows;
     for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
-      const ItemInfo it = decode_item(p, item);
+      const ItemInfo it = decode_item<kMode>(p, item);
       const int32_t *list = p.kv_list + ((long long)it.head * g.n_tiles + it.tile) * p.kv_stride;
       const int nbox = it.nc * pieces;  // K/V boxes of the item (K and V share coordinates)
       const bool staged = nbox <= kMaxCoords;
@@ -186,31 +192,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                           box_coords(p, it.bh, it.tile, off, off < g.tau), q_full);
             }
         }
-        // K and V chunks in the order the MMA uses them.  Shared chunks (one
-        // or two blocks): K0 V0 K1 V1 ...  Split item: K_A(0) K_B(0), then per
-        // step j: V_A(j) K_A(j+1) V_B(j) K_B(j+1), where warpgroup x's step j
-        // is chunk c0(x) + j.
-        auto emit = [&](int chunk, int is_v) -> bool {
-          const uint32_t slot = ld % C::kSlots, phase = (ld / C::kSlots) & 1;
-          if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrWaitProducer)) return false;
-          mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
-          uint8_t *dst = slots + slot * C::kTileBytes;
-          for (int pc = 0; pc < pieces; ++pc) {
-            const int e = chunk * pieces + pc;
-            load_box<D>(p, is_v ? &tmap_v : &tmap_k, dst + pc * p.piece_rows * 128,
-                        staged ? s_coord[e] : kv_coord(e), &full[slot]);
+        if constexpr (kMode == 0) {
+          // K and V chunks in the order the MMA first uses them: K0 V0 K1 V1 ...
+          for (int s = 0; s < 2 * it.nc && ok; ++s) {
+            const int chunk = s >> 1, is_v = s & 1;
+            const uint32_t slot = ld % C::kSlots, phase = (ld / C::kSlots) & 1;
+            if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrWaitProducer)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
+            uint8_t *dst = slots + slot * C::kTileBytes;
+            for (int pc = 0; pc < pieces; ++pc) {
+              const int e = chunk * pieces + pc;
+              load_box<D>(p, is_v ? &tmap_v : &tmap_k, dst + pc * p.piece_rows * 128,
+                          staged ? s_coord[e] : kv_coord(e), &full[slot]);
+            }
+            ++ld;
           }
-          ++ld;
-          return true;
-        };
-        const int nxk = it.split ? 2 : 1;  // K/V streams
-        for (int x = 0; x < nxk && ok; ++x) ok = emit(it.c0(x), 0);
-        for (int j = 0; j < it.n(0) && ok; ++j)
-          for (int x = 0; x < nxk && ok; ++x) {
-            if (j >= it.n(x)) continue;
-            ok = emit(it.c0(x) + j, 1);
-            if (ok && j + 1 < it.n(x)) ok = emit(it.c0(x) + j + 1, 0);
-          }
+        } else {
+          // Lone block: with one chunk, K0 V0.  Split: K_A(0) K_B(0), then per
+          // step j: V_A(j) K_A(j+1) V_B(j) K_B(j+1), warpgroup x's step j being
+          // chunk c0(x) + j.
+          auto emit = [&](int chunk, int is_v) -> bool {
+            const uint32_t slot = ld % C::kSlots, phase = (ld / C::kSlots) & 1;
+            if (!mbar_wait(&empty[slot], phase ^ 1, ctl, kErrWaitProducer)) return false;
+            mbar_arrive_expect_tx(&full[slot], C::kTileBytes);
+            uint8_t *dst = slots + slot * C::kTileBytes;
+            for (int pc = 0; pc < pieces; ++pc) {
+              const int e = chunk * pieces + pc;
+              load_box<D>(p, is_v ? &tmap_v : &tmap_k, dst + pc * p.piece_rows * 128,
+                          staged ? s_coord[e] : kv_coord(e), &full[slot]);
+            }
+            ++ld;
+            return true;
+          };
+          const int nxk = it.split ? 2 : 1;  // K/V streams
+          for (int x = 0; x < nxk && ok; ++x) ok = emit(it.c0(x), 0);
+          for (int j = 0; j < it.n(0) && ok; ++j)
+            for (int x = 0; x < nxk && ok; ++x) {
+              if (j >= it.n(x)) continue;
+              ok = emit(it.c0(x) + j, 1);
+              if (ok && j + 1 < it.n(x)) ok = emit(it.c0(x) + j + 1, 0);
+            }
+        }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       ld = __shfl_sync(0xffffffffu, ld, 0);
@@ -265,63 +287,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
 
-      for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
-        const ItemInfo it = decode_item(p, item);
-        const int nx = (it.has_b || it.split) ? 2 : 1;
-        const bool shared_kv = !it.split;  // block B reads block A's ring slots
-        if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t l = ld, kslot = 0, vslot = 0;
-        int s_left = it.nc;  // S groups still to issue (one per chunk)
-        // The ring slot for warpgroup x's next K or V: shared chunks reuse A's.
-        auto take = [&](int x, uint32_t &slot) -> bool {
-          if (x == 1 && shared_kv) return true;
-          if (!wait_slot(l)) return false;
-          slot = l++;
-          return true;
-        };
-        auto release = [&](int x, uint32_t slot) {
-          if (!shared_kv || x == nx - 1) mma_commit(&empty[slot % C::kSlots]);
-        };
-        auto s_group_done = [&](int x) {
-          if (shared_kv && x != nx - 1) return;
-          if (--s_left == 0) mma_commit(q_free);  // Q is no longer read
-        };
-        // first chunk of each warpgroup
-        for (int x = 0; x < nx && ok; ++x) {
-          if (!take(x, kslot)) { ok = false; break; }
-          mma_s(x, it.split ? 0 : x, kslot % C::kSlots);
+      if constexpr (kMode == 0)
+        for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
+          const ItemInfo it = decode_item<kMode>(p, item);
+          const int nx = it.has_b ? 2 : 1;
+          if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
+          tc_fence_after();
+          // chunk 0: S_A(0) [, S_B(0)]
+          const uint32_t k0 = ld;
+          if (!wait_slot(k0)) { ok = false; break; }
+          for (int x = 0; x < nx; ++x) mma_s(x, x, k0 % C::kSlots);
           issued = true;
-          release(x, kslot);
-          s_group_done(x);
-        }
-        for (int j = 0; j < it.n(0) && ok; ++j) {
-          for (int x = 0; x < nx; ++x) {
-            if (j >= it.n(x)) continue;
-            if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
-            ++p_waits[x];
-            tc_fence_after();
-            if (j == 0 && x_items[x] > 0) {
-              // the previous item of this warpgroup has read O_X in its epilogue
-              if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
-              ++o_waits[x];
+          mma_commit(&empty[k0 % C::kSlots]);
+          if (it.nc == 1) mma_commit(q_free);
+          for (int j = 0; j < it.nc && ok; ++j) {
+            const uint32_t vj = k0 + 2 * j + 1, kn = k0 + 2 * j + 2;  // V_j, K_{j+1} load indices
+            for (int x = 0; x < nx; ++x) {
+              if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+              ++p_waits[x];
               tc_fence_after();
-            }
-            if (!take(x, vslot)) { ok = false; break; }
-            mma_pv(x, vslot % C::kSlots, j == 0);
-            release(x, vslot);
-            if (j + 1 < it.n(x)) {
-              if (!take(x, kslot)) { ok = false; break; }
-              mma_s(x, it.split ? 0 : x, kslot % C::kSlots);
-              release(x, kslot);
-              s_group_done(x);
+              if (j == 0 && x_items[x] > 0) {
+                // the previous item of this block has read O_X in its epilogue
+                if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+                ++o_waits[x];
+                tc_fence_after();
+              }
+              if (x == 0 && !wait_slot(vj)) { ok = false; break; }
+              mma_pv(x, vj % C::kSlots, j == 0);
+              if (x == nx - 1) mma_commit(&empty[vj % C::kSlots]);
+              if (j + 1 < it.nc) {
+                if (x == 0 && !wait_slot(kn)) { ok = false; break; }
+                mma_s(x, x, kn % C::kSlots);
+                if (x == nx - 1) {
+                  mma_commit(&empty[kn % C::kSlots]);
+                  if (j + 2 == it.nc) mma_commit(q_free);
+                }
+              }
             }
           }
+          ld = k0 + 2 * it.nc;
+          for (int x = 0; x < nx; ++x) ++x_items[x];
+          ++item_ctr;
         }
-        ld = l;
-        for (int x = 0; x < nx; ++x) ++x_items[x];
-        ++item_ctr;
-      }
+      else
+        for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
+          const ItemInfo it = decode_item<kMode>(p, item);
+          const int nx = it.split ? 2 : 1;
+          if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t l = ld, kslot = 0, vslot = 0;
+          int s_left = it.nc;  // S groups still to issue (one per chunk)
+          // Each warpgroup has its own K/V stream: every chunk takes the next ring slot.
+          auto take = [&](uint32_t &slot) -> bool {
+            if (!wait_slot(l)) return false;
+            slot = l++;
+            return true;
+          };
+          auto release = [&](uint32_t slot) { mma_commit(&empty[slot % C::kSlots]); };
+          auto s_group_done = [&]() {
+            if (--s_left == 0) mma_commit(q_free);  // Q is no longer read
+          };
+          // first chunk of each warpgroup
+          for (int x = 0; x < nx && ok; ++x) {
+            if (!take(kslot)) { ok = false; break; }
+            mma_s(x, 0, kslot % C::kSlots);
+            issued = true;
+            release(kslot);
+            s_group_done();
+          }
+          for (int j = 0; j < it.n(0) && ok; ++j) {
+            for (int x = 0; x < nx; ++x) {
+              if (j >= it.n(x)) continue;
+              if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+              ++p_waits[x];
+              tc_fence_after();
+              if (j == 0 && x_items[x] > 0) {
+                // the previous item of this warpgroup has read O_X in its epilogue
+                if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+                ++o_waits[x];
+                tc_fence_after();
+              }
+              if (!take(vslot)) { ok = false; break; }
+              mma_pv(x, vslot % C::kSlots, j == 0);
+              release(vslot);
+              if (j + 1 < it.n(x)) {
+                if (!take(kslot)) { ok = false; break; }
+                mma_s(x, 0, kslot % C::kSlots);
+                release(kslot);
+                s_group_done();
+              }
+            }
+          }
+          ld = l;
+          for (int x = 0; x < nx; ++x) ++x_items[x];
+          ++item_ctr;
+        }
       if (!ok && issued) {
         // Wait for every MMA already issued before TMEM is released.
         mma_commit(drain);
@@ -343,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // named barriers of split items.
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_work; item += gridDim.x) {
-      const ItemInfo it = decode_item(p, item);
+      const ItemInfo it = decode_item<kMode>(p, item);
       if (it.n(x) == 0) continue;
       const int o_in_tile = (it.qa + (it.split ? 0 : x)) * kBM + row;
       const bool row_valid = o_in_tile < g.tau;
@@ -524,21 +584,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_fwd_d(const FwdParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                         int num_sms, cudaStream_t stream) {
+template <int D, int kMode>
+cudaError_t launch_fwd_mode(const FwdParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            int num_sms, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static bool attr_set = false;  // per process; the attribute is per function
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(sta_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(sta_fwd_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int grid = p.n_work < num_sms ? p.n_work : num_sms;
   if (grid <= 0) return cudaSuccess;
-  sta_fwd_kernel<D><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  sta_fwd_kernel<D, kMode><<<grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+// The work list holds the items of one or two shared blocks first and the
+// lone blocks (n_work_lone of them) last; each part gets its own launch.
+template <int D>
+cudaError_t launch_fwd_d(const FwdParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         int num_sms, cudaStream_t stream) {
+  FwdParams part = p;
+  part.n_work = p.n_work - p.n_work_lone;
+  cudaError_t e = launch_fwd_mode<D, 0>(part, tq, tk, tv, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  part.work = p.work + part.n_work;
+  part.n_work = p.n_work_lone;
+  return launch_fwd_mode<D, 1>(part, tq, tk, tv, num_sms, stream);
 }
 
 }  // namespace

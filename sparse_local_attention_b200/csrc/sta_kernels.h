@@ -44,8 +44,9 @@ struct FwdParams {
   const int32_t *kv_list;   // [Hh][n_tiles][kv_stride]
   const int32_t *kv_count;  // [Hh]
   int kv_stride;
-  const int2 *work;  // (bh, tile * npairs + pair), heaviest first
+  const int2 *work;  // (bh, tile * npairs + pair), heaviest first within each kind
   int n_work;
+  int n_work_lone;   // the last n_work_lone items hold one query block (the one-CTA kernel)
   float scale_log2;  // softmax scale * log2(e)
   int *status;       // device status word
   unsigned long long wait_limit_ns;

@@ -28,7 +28,7 @@ STA_CALL_CHECK = 0x1
 
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
             "sta_plan_q_tiles", "sta_plan_geometry", "sta_permute", "sta_forward", "sta_backward",
-            "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc"]
+            "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc", "sta_plan_launches"]
 
 
 class StaError(RuntimeError):
@@ -147,6 +147,9 @@ class Plan:
         nt, tv = ctypes.c_int32(), ctypes.c_int32()
         _check(lib().sta_plan_geometry(handle, ctypes.byref(nt), ctypes.byref(tv)), "sta_plan_geometry")
         self.n_tiles, self.tile_volume = nt.value, tv.value
+        fl, bl = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().sta_plan_launches(handle, ctypes.byref(fl), ctypes.byref(bl)), "sta_plan_launches")
+        self.forward_launches, self.backward_launches = fl.value, bl.value  # kernels per call
 
     def destroy(self):
         if self.handle is not None and self.handle.value:
