@@ -5,10 +5,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <new>
 #include <numeric>
 #include <vector>
@@ -28,10 +30,10 @@ struct sta_plan_s {
   std::vector<int32_t> kv_list;  // [heads][n_tiles][kv_stride]
   std::vector<int32_t> inv_off;  // [heads][n_tiles + 1], absolute into inv_idx
   std::vector<int32_t> inv_idx;
-  std::vector<int2> work;        // forward work items
+  std::vector<int4> work;        // forward work items (see FwdParams::work)
   std::vector<int2> work_kv;     // backward dK/dV items (bh, key tile * nqb + key block)
   std::vector<int2> work_q;      // backward dQ items (bh, query tile * nqb + query block)
-  int npairs = 1;
+  int nqb = 1;  // 128-row query blocks per tile
   int n_work_lone = 0;  // forward items with one query block, at the end of `work`
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
@@ -43,7 +45,8 @@ struct sta_plan_s {
   int device = -1, num_sms = 0;
   // device copies
   int32_t *d_kv_list = nullptr, *d_count = nullptr, *d_inv_off = nullptr, *d_inv_idx = nullptr;
-  int2 *d_work = nullptr, *d_work_kv = nullptr, *d_work_q = nullptr;
+  int4 *d_work = nullptr;
+  int2 *d_work_kv = nullptr, *d_work_q = nullptr;
 };
 
 namespace {
@@ -161,7 +164,8 @@ void free_device(sta_plan_s *pl) {
   cudaFree(pl->d_work_kv);
   cudaFree(pl->d_work_q);
   pl->d_kv_list = pl->d_count = pl->d_inv_off = pl->d_inv_idx = nullptr;
-  pl->d_work = pl->d_work_kv = pl->d_work_q = nullptr;
+  pl->d_work = nullptr;
+  pl->d_work_kv = pl->d_work_q = nullptr;
 }
 
 template <class T>
@@ -264,7 +268,7 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
   g.n_tiles = g.GT * g.GH * g.GW;
   g.tau = (int)tau;
   pl->scale = prob->scale > 0.f ? prob->scale : 1.0f / std::sqrt((float)g.d);
-  pl->npairs = (g.tau + 255) / 256;
+  pl->nqb = (g.tau + 127) / 128;
 
   try {
     // --- per-head clamped windows and list lengths
@@ -320,38 +324,67 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       }
     }
 
-    // --- forward work items: pairs of 128-row query blocks of one tile (the
-    //     last item of a tile with an odd number of blocks has one block).
-    //     The persistent grid takes items round-robin, so they are ordered by
-    //     cost, largest first (query blocks x key tiles: a longest-processing-
-    //     time order); within a cost, head by head and tile by tile, so
-    //     consecutive items share most of their key tiles in L2.  The lone
-    //     blocks then move to the end: the one-CTA forward runs them as a
-    //     launch of their own (a grid stride over mixed kinds would hand some
-    //     CTAs only two-block items and others only lone blocks).
+    // --- forward work items: pairs of 128-row query blocks that attend to the
+    //     same key tiles, so that each K/V chunk brought in serves 256 rows.
+    //     Blocks 2i, 2i+1 of a tile pair up.  When a tile has an odd number of
+    //     blocks, its last block pairs with the last block of another tile of
+    //     the same head whose KV-tile list is the same (tiles whose clamped
+    //     windows coincide, as they do next to the grid borders); a block left
+    //     without such a partner is a lone item.  Lone items go last: the
+    //     one-CTA forward runs them as a launch of their own.  Within each
+    //     kind the persistent grid takes items round-robin, so they are ordered
+    //     by cost, largest first (query blocks x key tiles: a longest-
+    //     processing-time order); within a cost, head by head and tile by tile,
+    //     so consecutive items share most of their key tiles in L2.
     std::vector<int> heads(g.Hh);
     std::iota(heads.begin(), heads.end(), 0);
     std::stable_sort(heads.begin(), heads.end(), [&](int a, int b) { return pl->count[a] > pl->count[b]; });
-    pl->work.reserve((size_t)g.B * g.Hh * g.n_tiles * pl->npairs);
-    for (int h : heads)
-      for (int b = 0; b < g.B; ++b)
-        for (int t = 0; t < g.n_tiles; ++t)
-          for (int pr = 0; pr < pl->npairs; ++pr) pl->work.push_back(make_int2(b * g.Hh + h, t * pl->npairs + pr));
-    {
-      const int nqb = (g.tau + 127) / 128;
-      auto cost = [&](const int2 &w) {
-        const int pr = w.y % pl->npairs;
-        return (long long)std::min(2, nqb - 2 * pr) * pl->count[w.x % g.Hh];
-      };
-      std::stable_sort(pl->work.begin(), pl->work.end(), [&](const int2 &a, const int2 &b) { return cost(a) > cost(b); });
-      // items with a lone query block last (the one-CTA forward launches them separately)
-      auto lone = [&](const int2 &w) { return 2 * (w.y % pl->npairs) + 1 == nqb; };
-      auto mid = std::stable_partition(pl->work.begin(), pl->work.end(), [&](const int2 &w) { return !lone(w); });
-      pl->n_work_lone = (int)(pl->work.end() - mid);
+    const int nqb = pl->nqb;
+    std::vector<int4> lone_items;
+    std::vector<int> partner(g.n_tiles);
+    for (int h : heads) {
+      // partner[t]: the tile whose last block shares an item with t's last block
+      // (t itself when t leads such an item, -1 when t's last block is lone,
+      // -2 when t's last block is taken by an earlier tile)
+      std::fill(partner.begin(), partner.end(), -1);
+      if (nqb % 2 == 1) {
+        const int *w = &pl->wclamp[3 * h];
+        std::map<std::array<int, 3>, int> open;  // window start -> tile waiting for a partner
+        for (int t = 0; t < g.n_tiles; ++t) {
+          const int qt = t / (g.GH * g.GW), qh = (t / g.GW) % g.GH, qw = t % g.GW;
+          const std::array<int, 3> key = {window_start(qt, w[0], g.GT), window_start(qh, w[1], g.GH),
+                                          window_start(qw, w[2], g.GW)};
+          auto f = open.find(key);
+          if (f == open.end()) {
+            open[key] = t;
+          } else {
+            partner[f->second] = t;
+            partner[t] = -2;
+            open.erase(f);
+          }
+        }
+      }
+      for (int b = 0; b < g.B; ++b) {
+        const int bh = b * g.Hh + h;
+        for (int t = 0; t < g.n_tiles; ++t) {
+          for (int qb = 0; qb + 1 < nqb; qb += 2)
+            pl->work.push_back(make_int4(bh, t * nqb + qb, t * nqb + qb + 1, 0));
+          if (nqb % 2 == 1) {
+            const int last = t * nqb + nqb - 1;
+            if (partner[t] >= 0) pl->work.push_back(make_int4(bh, last, partner[t] * nqb + nqb - 1, 0));
+            else if (partner[t] == -1) lone_items.push_back(make_int4(bh, last, -1, 0));
+          }
+        }
+      }
     }
+    auto cost = [&](const int4 &w) { return (long long)(w.z >= 0 ? 2 : 1) * pl->count[w.x % g.Hh]; };
+    auto by_cost = [&](const int4 &a, const int4 &b) { return cost(a) > cost(b); };
+    std::stable_sort(pl->work.begin(), pl->work.end(), by_cost);
+    std::stable_sort(lone_items.begin(), lone_items.end(), by_cost);
+    pl->n_work_lone = (int)lone_items.size();
+    pl->work.insert(pl->work.end(), lone_items.begin(), lone_items.end());
 
     if (prob->flags & STA_PROBLEM_BACKWARD) {
-      const int nqb = (g.tau + 127) / 128;
       // dQ: one 128-row query block per item, heaviest heads first.
       for (int h : heads)
         for (int b = 0; b < g.B; ++b)
@@ -552,7 +585,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   fp.g = pl->g;
   fp.q = q, fp.o = o, fp.lse = lse;
   fp.tiled = pl->tiled ? 1 : 0;
-  fp.npairs = pl->npairs;
+  fp.nqb = pl->nqb;
   fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
   fp.work = pl->d_work, fp.n_work = (int)pl->work.size(), fp.n_work_lone = pl->n_work_lone;
   fp.scale_log2 = pl->scale * 1.4426950408889634f;

@@ -7,15 +7,16 @@
 //
 // Design (B200):
 //   * persistent grid, one CTA per SM.  A work item is a pair of 128-row
-//     query blocks (A, B) of the same query tile -- both attend to the same
-//     key tiles, so every K/V chunk brought into shared memory serves 256
-//     query rows.  When a tile has an odd number of blocks the last item has
-//     one block; its key chunks are then divided between the two warpgroups
-//     (the first half to A, the rest to B, both reading the same Q) and the
-//     epilogue merges the two partial softmax states, so a lone block still
-//     keeps two MMA/softmax chains in flight.  The two kinds of item run as
-//     two launches of two instantiations (kMode 0 / 1), each over its part of
-//     the work list, heaviest items first.
+//     query blocks (A, B) that attend to the same key tiles -- two blocks of
+//     one query tile, or the last blocks of two tiles whose windows coincide
+//     -- so every K/V chunk brought into shared memory serves 256 query rows.
+//     A block left without a partner is a lone item; its key chunks are
+//     divided between the two warpgroups (the first half to A, the rest to
+//     B, both reading the same Q) and the epilogue merges the two partial
+//     softmax states, so a lone block still keeps two MMA/softmax chains in
+//     flight.  The two kinds of item run as two launches of two
+//     instantiations (kMode 0 / 1), each over its part of the work list,
+//     heaviest items first.
 //   * warp 8: TMA producer.  Loads Q_A, Q_B (shared memory, 128-byte swizzle)
 //     and streams K and V chunks of 128 keys into a ring of stages, gathering
 //     them tile by tile from the KV-tile list.  At the start of an item the
@@ -51,12 +52,14 @@ constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kMaxCoords = 1024;  // per-item K/V box coordinates staged in shared memory
 
-template <int D>
+template <int D, int kMode>
 struct FwdCfg {
   static constexpr uint32_t kPanelBytes = kBN * 128;  // 128 rows x 64 bf16
   static constexpr uint32_t kTileBytes = kBN * D * 2;  // one Q block or one K / V chunk
-  static constexpr int kPanels = D / 64;
-  static constexpr int kSlots = D == 128 ? 4 : 8;
+  static constexpr int kNumQ = kMode == 0 ? 2 : 1;     // Q blocks held (a lone block needs one)
+  // K/V ring: what shared memory holds besides Q; a lone block's second K/V
+  // stream gets the space of the Q block it does not need
+  static constexpr int kSlots = (D == 128 ? 4 : 8) + (2 - kNumQ);
   static constexpr uint32_t kTmO0 = 256;  // O_X at kTmO0 + X * D; S_X at 128 * X
   static constexpr uint32_t kTmCols = 512;
   // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain
@@ -64,13 +67,14 @@ struct FwdCfg {
   static constexpr uint32_t kMiscBytes = 64 + 4 * 128 * 4;  // tmem address, abort flag, m/l exchange
   static constexpr uint32_t kListBytes = kMaxCoords * 16;
   static constexpr uint32_t kSmemBytes =
-      (2 + kSlots) * kTileBytes + kNumBars * 8 + kMiscBytes + 16 + kListBytes + 1024;
+      (kNumQ + kSlots) * kTileBytes + kNumBars * 8 + kMiscBytes + 16 + kListBytes + 1024;
   static_assert(kTmO0 + 2 * D <= kTmCols, "TMEM budget");
 };
 
 struct ItemInfo {
-  int bh, tile, head, qa;  // qa = first query block of the pair
-  bool has_b;              // a second query block (qa + 1) shares the K/V chunks
+  int bh, head, tile;      // tile: whose KV-tile list the item walks (block A's)
+  int ta, qa, tb, qb;      // query block A = block qa of tile ta; B = block qb of tile tb
+  bool has_b;              // a second query block shares the K/V chunks
   bool split;              // one query block, its chunks divided between the two warpgroups
   int nkeys, nc;
   int n0, n1, c1;          // chunks of warpgroup 0: 0 .. n0 - 1; of warpgroup 1: c1 .. c1 + n1 - 1
@@ -84,13 +88,16 @@ struct ItemInfo {
 // work list, so that each instantiation carries only the code it runs.
 template <int kMode>
 __device__ __forceinline__ ItemInfo decode_item(const FwdParams &p, int item) {
-  const int2 wi = p.work[item];
+  const int4 wi = p.work[item];
   ItemInfo it;
   it.bh = wi.x;
-  it.tile = wi.y / p.npairs;
-  it.qa = 2 * (wi.y % p.npairs);
+  it.ta = wi.y / p.nqb;
+  it.qa = wi.y - it.ta * p.nqb;
+  it.has_b = kMode == 0 && wi.z >= 0;
+  it.tb = it.has_b ? wi.z / p.nqb : it.ta;
+  it.qb = it.has_b ? wi.z - it.tb * p.nqb : it.qa;
+  it.tile = it.ta;
   it.head = it.bh % p.g.Hh;
-  it.has_b = kMode == 0 && (it.qa + 1) * kBM < p.g.tau;
   it.nkeys = p.kv_count[it.head] * p.g.tau;
   it.nc = (it.nkeys + kBN - 1) / kBN;
   it.split = kMode == 1 && it.nc > 1;
@@ -104,11 +111,11 @@ template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     sta_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kMode>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *q_smem = smem;                                  // [2][D/64 panels][128 rows][64]
-  uint8_t *slots = smem + 2 * C::kTileBytes;               // [kSlots][D/64][128][64]
+  uint8_t *q_smem = smem;                                  // [kNumQ][D/64 panels][128 rows][64]
+  uint8_t *slots = smem + C::kNumQ * C::kTileBytes;        // [kSlots][D/64][128][64]
   uint64_t *bars = reinterpret_cast<uint64_t *>(slots + C::kSlots * C::kTileBytes);
   uint64_t *full = bars;
   uint64_t *empty = bars + C::kSlots;
@@ -187,9 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(q_full, (it.has_b ? 2 : 1) * C::kTileBytes);
           for (int x = 0; x < (it.has_b ? 2 : 1); ++x)
             for (int pc = 0; pc < pieces; ++pc) {
-              const int off = (it.qa + x) * kBM + pc * p.piece_rows;
+              const int off = (x ? it.qb : it.qa) * kBM + pc * p.piece_rows;
               load_box<D>(p, &tmap_q, q_smem + x * C::kTileBytes + pc * p.piece_rows * 128,
-                          box_coords(p, it.bh, it.tile, off, off < g.tau), q_full);
+                          box_coords(p, it.bh, x ? it.tb : it.ta, off, off < g.tau), q_full);
             }
         }
         if constexpr (kMode == 0) {
@@ -225,12 +232,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             return true;
           };
           const int nxk = it.split ? 2 : 1;  // K/V streams
-          for (int x = 0; x < nxk && ok; ++x) ok = emit(it.c0(x), 0);
-          for (int j = 0; j < it.n(0) && ok; ++j)
-            for (int x = 0; x < nxk && ok; ++x) {
-              if (j >= it.n(x)) continue;
-              ok = emit(it.c0(x) + j, 1);
-              if (ok && j + 1 < it.n(x)) ok = emit(it.c0(x) + j + 1, 0);
+          // step -1 loads each stream's first K; step j >= 0 its V(j), then K(j + 1)
+#pragma unroll 1
+          for (int st = -1; st < it.n0 && ok; ++st)
+#pragma unroll 1
+            for (int e = 0; e < 2 * nxk && ok; ++e) {
+              const int x = e >> 1, is_v = (e & 1) ^ 1;
+              const int j = is_v ? st : st + 1;  // step of the chunk this load serves
+              if ((st < 0 && is_v) || j >= it.n(x)) continue;
+              ok = emit(it.c0(x) + j, is_v);
             }
         }
       }
@@ -405,9 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int item = blockIdx.x; item < p.n_work; item += gridDim.x) {
       const ItemInfo it = decode_item<kMode>(p, item);
       if (it.n(x) == 0) continue;
-      const int o_in_tile = (it.qa + (it.split ? 0 : x)) * kBM + row;
+      const bool own_b = x == 1 && !it.split;  // warpgroup 1 holds block B
+      const int o_in_tile = (own_b ? it.qb : it.qa) * kBM + row;
       const bool row_valid = o_in_tile < g.tau;
-      const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, o_in_tile) : 0;
+      const long long tok = row_valid ? token_row(g, p.tiled, it.bh, own_b ? it.tb : it.ta, o_in_tile) : 0;
 
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < it.n(x) && ok; ++j) {
@@ -587,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int kMode>
 cudaError_t launch_fwd_mode(const FwdParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             int num_sms, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kMode>;
   static bool attr_set = false;  // per process; the attribute is per function
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(sta_fwd_kernel<D, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -49,15 +49,18 @@ constexpr uint32_t kSmemBytes = kSlots * kSlotBytes + kNumBars * 8 + kMiscBytes 
                                 kMaxCoords * 16 + 1024;
 
 struct PairItem {
-  int bh, tile, head, qa, nkeys, nc;
+  int bh, tile, head, nkeys, nc;  // tile: whose KV-tile list the item walks
+  int my_tile, my_qb;             // this CTA's query block (my_qb == -1: none)
 };
 
 __device__ __forceinline__ PairItem decode_pair(const FwdParams &p, int item) {
-  const int2 wi = p.work[item];
+  const int4 wi = p.work[item];
   PairItem it;
   it.bh = wi.x;
-  it.tile = wi.y / p.npairs;
-  it.qa = 2 * (wi.y % p.npairs);
+  it.tile = wi.y / p.nqb;
+  const int mine = cluster_ctarank() ? wi.z : wi.y;
+  it.my_tile = mine >= 0 ? mine / p.nqb : it.tile;
+  it.my_qb = mine >= 0 ? mine - it.my_tile * p.nqb : -1;
   it.head = it.bh % p.g.Hh;
   it.nkeys = p.kv_count[it.head] * p.g.tau;
   it.nc = (it.nkeys + kBN - 1) / kBN;
@@ -276,9 +279,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int item = cid; item < p.n_work && ok; item += ncl) {
       const PairItem it = decode_pair(p, item);
-      const int o_in_tile = (it.qa + (int)rank) * kBM + row;
-      const bool row_valid = o_in_tile < g.tau;
-      const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, o_in_tile) : 0;
+      const int o_in_tile = it.my_qb * kBM + row;  // negative when this CTA has no block
+      const bool row_valid = it.my_qb >= 0 && o_in_tile < g.tau;
+      const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.my_tile, o_in_tile) : 0;
       {
         // Q row -> TMEM; warpgroup wg writes elements [64 wg, 64 wg + 64)
         const uint4 *src =

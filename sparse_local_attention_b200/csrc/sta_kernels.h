@@ -40,13 +40,17 @@ struct FwdParams {
   void *o;           // bf16
   float *lse;        // fp32, nullable
   int tiled;         // q / o / lse are tile-major instead of raster
-  int npairs;        // work items per tile: pairs of 128-row query blocks = ceil(tau / 256)
+  int nqb;           // 128-row query blocks per tile = ceil(tau / 128)
   const int32_t *kv_list;   // [Hh][n_tiles][kv_stride]
   const int32_t *kv_count;  // [Hh]
   int kv_stride;
-  const int2 *work;  // (bh, tile * npairs + pair), heaviest first within each kind
+  // Work items (bh, a, b, 0): query block A = a % nqb of tile a / nqb and query
+  // block B likewise from b, or b = -1 for a lone block.  A and B attend to the
+  // same key tiles (the KV-tile list of A's tile).  Heaviest first within each
+  // kind; the last n_work_lone items are the lone blocks.
+  const int4 *work;
   int n_work;
-  int n_work_lone;   // the last n_work_lone items hold one query block (the one-CTA kernel)
+  int n_work_lone;
   float scale_log2;  // softmax scale * log2(e)
   int *status;       // device status word
   unsigned long long wait_limit_ns;

@@ -70,16 +70,17 @@ def test_backward_requires_backward_tables():
         sta.sta_plan_q_tiles(plan, 0)
 
 
-@pytest.mark.parametrize("tile,T,H,W,forward", [
-    ((4, 8, 8), 8, 16, 16, 1),   # 256 tokens: two query blocks per tile, one kind of item
-    ((6, 8, 8), 12, 16, 16, 2),  # 384 tokens: a block pair and a lone block per tile
-    ((2, 4, 4), 4, 8, 8, 1),     # 32 tokens: lone blocks only
-    ((2, 6, 4), 4, 12, 8, 4),    # 48 tokens, not a box of the raster tensor: 3 gathers + lone blocks
+@pytest.mark.parametrize("tile,T,H,W,win,forward", [
+    ((4, 8, 8), 8, 16, 16, (3, 3, 3), 1),   # 256 tokens: two query blocks per tile
+    ((6, 8, 8), 12, 16, 16, (3, 3, 3), 1),  # 384 tokens, one window for all tiles: last blocks pair up
+    ((6, 8, 8), 6, 8, 24, (1, 1, 1), 2),    # 384 tokens, every window distinct: lone last blocks
+    ((2, 4, 4), 4, 8, 8, (3, 3, 3), 1),     # 32 tokens: one block per tile, paired across tiles
+    ((2, 6, 4), 4, 12, 8, (3, 3, 3), 4),    # 48 tokens, not a box of the raster tensor: 3 gathers + pairs
 ])
-def test_plan_launch_counts(tile, T, H, W, forward):
-    plan = _create(head_dim=128, T=T, H=H, W=W, tile=tile, windows=[(3, 3, 3)], backward=True)
+def test_plan_launch_counts(tile, T, H, W, win, forward):
+    plan = _create(head_dim=128, T=T, H=H, W=W, tile=tile, windows=[win], backward=True)
     assert plan.forward_launches == forward
     gather = forward == 4
     assert plan.backward_launches == (4 if gather else 0) + 3
-    plan_f = _create(head_dim=128, T=T, H=H, W=W, tile=tile, windows=[(3, 3, 3)])
+    plan_f = _create(head_dim=128, T=T, H=H, W=W, tile=tile, windows=[win])
     assert plan_f.backward_launches == 0
