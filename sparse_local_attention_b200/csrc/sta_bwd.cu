@@ -13,15 +13,20 @@
 //   2. bwd_dkdv: one 128-row key block per work item (key-block major).  K and
 //      V stay in shared memory; the query blocks of every query tile whose
 //      window holds the key tile (the planner's inverse lists) stream through
-//      a ring.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the softmax warps
-//      (thread = key row) turn them into P^T and dS^T (bf16, written over the
-//      consumed columns), then dV += P^T dO and dK += dS^T Q accumulate in
-//      TMEM with P^T / dS^T as the TMEM A operand.
+//      a ring.  S^T = K Q^T and dP^T = V dO^T land in TMEM; the elementwise
+//      warps (thread = key row) turn them into P^T and dS^T (bf16), then
+//      dV += P^T dO and dK += dS^T Q accumulate in TMEM with P^T / dS^T as the
+//      TMEM A operand.  With head dim 64, P^T / dS^T have TMEM columns of their
+//      own and S^T / dP^T of the next query chunk are computed while the
+//      elementwise warps work; with head dim 128 they are written over the
+//      columns they come from.
 //   3. bwd_dq: one 128-row query block per work item (query-block major, the
 //      forward KV-tile lists).  S = Q K^T and dP = dO V^T per 128-key chunk,
-//      dS in TMEM, dQ += dS K.
-// Warp roles as in the forward: warps 0-3 elementwise math (thread = TMEM
-// lane = row), warp 4 TMA producer, warp 5 MMA issuer.  Every wait is bounded.
+//      dS in TMEM columns of its own, dQ += dS K; the next chunk's S / dP are
+//      computed while the elementwise warps work on this one.
+// Warp roles as in the forward: warps 0-7 elementwise math in two warpgroups
+// that split each chunk's columns (thread = TMEM lane = row), warp 8 TMA
+// producer, warp 9 MMA issuer.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -32,8 +37,9 @@ namespace sta {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4, kMmaWarp = 5;
+constexpr int kThreads = 320;  // 8 elementwise warps, producer, MMA issuer
+constexpr int kMathWarps = 8;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kMaxCoords = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -78,15 +84,26 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 }
 
 // ----------------------------------------------------------------------- 2. dK, dV
+// Warps 0-7 elementwise (warpgroup e = query columns [64 e, 64 e + 64) of each
+// 128-query chunk; thread = key row = TMEM lane), warp 8 TMA producer, warp 9
+// MMA issuer.  With head dim 64, P^T and dS^T get TMEM columns of their own,
+// so S^T / dP^T of chunk i + 1 are computed while the elementwise warps work
+// on chunk i; with head dim 128 the accumulators leave no room and P^T / dS^T
+// are written over the S^T / dP^T columns they come from.
 template <int D>
 struct DkvCfg {
   static constexpr uint32_t kTile = kBM * D * 2;           // one 128-row operand tile
   static constexpr uint32_t kPanel = kBM * 128;
+  static constexpr bool kSep = D == 64;                    // P^T, dS^T in columns of their own
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr uint32_t kStage = 2 * kTile + 1024;     // Q, dO, LSE2[128], D[128]
-  static constexpr int kNumBars = 2 * kStages + 7;
+  // barriers: st_full[S] st_empty[S] kv_full kv_free s_full s_read p_ready pd_free acc_done acc_free drain
+  static constexpr int kNumBars = 2 * kStages + 9;
   static constexpr uint32_t kSmem = 2 * kTile + kStages * kStage + kNumBars * 8 + 64 + 1024;
-  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 256 + D;
+  static constexpr uint32_t kTmS = 0, kTmDP = 128;
+  static constexpr uint32_t kTmP = kSep ? 256 : kTmS, kTmDS = kSep ? 320 : kTmDP;
+  static constexpr uint32_t kTmDV = kSep ? 384 : 256, kTmDK = kTmDV + D;
+  static_assert(kTmDK + D <= 512, "TMEM budget");
 };
 
 template <int D>
@@ -101,8 +118,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, lse2[128], dd[128]}
   uint64_t *bars = reinterpret_cast<uint64_t *>(stages + C::kStages * C::kStage);
   uint64_t *st_full = bars, *st_empty = bars + C::kStages;
-  uint64_t *kv_full = bars + 2 * C::kStages, *kv_free = kv_full + 1, *s_full = kv_full + 2, *p_ready = kv_full + 3;
-  uint64_t *acc_done = kv_full + 4, *acc_free = kv_full + 5, *drain = kv_full + 6;
+  uint64_t *kv_full = bars + 2 * C::kStages, *kv_free = kv_full + 1;
+  uint64_t *s_full = kv_full + 2;    // S^T, dP^T of a chunk are in TMEM
+  uint64_t *s_read = kv_full + 3;    // ... and have been read (separate P / dS columns only)
+  uint64_t *p_ready = kv_full + 4;   // P^T, dS^T written
+  uint64_t *pd_free = kv_full + 5;   // the dV / dK MMAs have read them (separate columns only)
+  uint64_t *acc_done = kv_full + 6, *acc_free = kv_full + 7, *drain = kv_full + 8;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -116,9 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(kv_full, 1);
     mbar_init(kv_free, 1);
     mbar_init(s_full, 1);
-    mbar_init(p_ready, 4);
+    mbar_init(s_read, kMathWarps);
+    mbar_init(p_ready, kMathWarps);
+    mbar_init(pd_free, 1);
     mbar_init(acc_done, 1);
-    mbar_init(acc_free, 4);
+    mbar_init(acc_free, kMathWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -193,50 +216,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t kd = smem_desc_sw128(smem_u32(k_s), 16, 1024), vd = smem_desc_sw128(smem_u32(v_s), 16, 1024);
       const uint64_t sk0 = smem_desc_sw128(smem_u32(stages), 16, 1024);              // K-major Q / dO
       const uint64_t sm0 = smem_desc_sw128(smem_u32(stages), C::kPanel, 1024);       // MN-major Q / dO
-      uint32_t ld = 0, item_ctr = 0, p_waits = 0;
+      uint32_t ld = 0, item_ctr = 0, p_waits = 0, r_waits = 0;
       bool ok = true, issued = false;
+      // S^T = K Q^T and dP^T = V dO^T for the chunk in stage `st`
+      auto issue_s = [&](uint32_t st) {
+        const uint32_t so = (st * C::kStage) >> 4, dso = (st * C::kStage + C::kTile) >> 4;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+      };
+      auto wait_stage = [&](uint32_t l) -> bool {
+        if (!mbar_wait(&st_full[l % C::kStages], (l / C::kStages) & 1, ctl, kErrBwdWait)) return false;
+        tc_fence_after();
+        return true;
+      };
       for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
         int bh, ktile, kb, off0, nq;
         item_info(item, bh, ktile, kb, off0, nq);
         if (!mbar_wait(kv_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
         tc_fence_after();
+        if (!wait_stage(ld)) { ok = false; break; }
+        issue_s(ld % C::kStages);
+        issued = true;
         for (int i = 0; i < nq && ok; ++i) {
-          const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
-          if (!mbar_wait(&st_full[st], ph, ctl, kErrBwdWait)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t so = (st * C::kStage) >> 4, dso = (st * C::kStage + C::kTile) >> 4;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
+          const uint32_t cur = ld + i, st = cur % C::kStages;
+          if (C::kSep && i + 1 < nq) {
+            // the next chunk's S^T / dP^T as soon as this chunk's have been read
+            if (!mbar_wait(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+            ++r_waits;
+            tc_fence_after();
+            if (!wait_stage(cur + 1)) { ok = false; break; }
+            issue_s((cur + 1) % C::kStages);
           }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
-          }
-          issued = true;
-          mma_commit(s_full);
-          if (i == nq - 1) mma_commit(kv_free);
           if (!mbar_wait(p_ready, p_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
           ++p_waits;
           if (i == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO and dK += dS^T Q (queries are the contraction, 8 steps of 16)
+          const uint32_t so = (st * C::kStage) >> 4, dso = (st * C::kStage + C::kTile) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             const uint32_t off = (kk * 16 * 128) >> 4;
-            mma_ts(tmem + C::kTmDV, tmem + C::kTmS + kk * 8, sm0 + dso + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + C::kTmDV, tmem + C::kTmP + kk * 8, sm0 + dso + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             const uint32_t off = (kk * 16 * 128) >> 4;
-            mma_ts(tmem + C::kTmDK, tmem + C::kTmDP + kk * 8, sm0 + so + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + C::kTmDK, tmem + C::kTmDS + kk * 8, sm0 + so + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&st_empty[st]);
-          ++ld;
+          if (C::kSep) mma_commit(pd_free);
+          if (i + 1 == nq) mma_commit(kv_free);
+          if (!C::kSep && i + 1 < nq) {
+            // P^T / dS^T live in the S^T / dP^T columns: the next S^T / dP^T
+            // are issued after the MMAs that read them (in-order execution)
+            if (!wait_stage(cur + 1)) { ok = false; break; }
+            issue_s((cur + 1) % C::kStages);
+          }
         }
         if (!ok) break;
+        ld += nq;
         mma_commit(acc_done);
         ++item_ctr;
       }
@@ -246,84 +293,111 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // elementwise warps: thread = key row of the block = TMEM lane
-    const int row = warp * 32 + lane;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    // elementwise warps: thread = key row of the block = TMEM lane; warpgroup
+    // e owns query columns [64 e, 64 e + 64)
+    const int e = warp >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const float sl2 = p.scale_log2;
-    uint32_t ld = 0, s_waits = 0, item_ctr = 0;
+    uint32_t ld = 0, s_waits = 0, f_waits = 0, item_ctr = 0, gchunk = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
       int bh, ktile, kb, off0, nq;
       item_info(item, bh, ktile, kb, off0, nq);
       const int krow = kb * kBM + row;
       const bool row_valid = krow < g.tau;
-      for (int i = 0; i < nq; ++i) {
+      for (int i = 0; i < nq; ++i, ++gchunk) {
         const int qb = i % p.nqb;
         const int valid_q = min(kBM, g.tau - qb * kBM);
         const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
         bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
-        if (!okw) { ok = false; break; }
-        tc_fence_after();
-        const float *lse_s = reinterpret_cast<const float *>(stages + st * C::kStage + 2 * C::kTile);
+        // two halves of 32 columns: load, then turn into packed P^T / dS^T
+        const float *lse_s = reinterpret_cast<const float *>(stages + st * C::kStage + 2 * C::kTile) + 64 * e;
         const float *dd_s = lse_s + 128;
+        uint32_t pp[2][16], pd[2][16];
 #pragma unroll
-        for (int c = 0; c < kBM / 32; ++c) {
+        for (int hf = 0; hf < 2; ++hf) {
           uint32_t rs[32], rd[32];
-          tmem_ld32(tmem + lane_off + C::kTmS + c * 32, rs);
-          tmem_ld32(tmem + lane_off + C::kTmDP + c * 32, rd);
-          tmem_ld_wait();
-          uint32_t pp[16], pd[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int q = c * 32 + e;
-            float pr[2], dr[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const bool v = q + h < valid_q;
-              const float pv = ex2_approx(fmaf(__uint_as_float(rs[e + h]), sl2, -lse_s[q + h]));
-              pr[h] = v ? pv : 0.f;
-              dr[h] = v ? pv * (__uint_as_float(rd[e + h]) - dd_s[q + h]) : 0.f;
-            }
-            pp[e / 2] = pack_bf16(pr[0], pr[1]);
-            pd[e / 2] = pack_bf16(dr[0], dr[1]);
+          if (okw) {
+            if (hf == 0) tc_fence_after();
+            const uint32_t base = tmem + lane_off + 64 * e + 32 * hf;
+            tmem_ld32(base + C::kTmS, rs);
+            tmem_ld32(base + C::kTmDP, rd);
+            tmem_ld_wait();
           }
-          tmem_st16(tmem + lane_off + C::kTmS + c * 16, pp);
-          tmem_st16(tmem + lane_off + C::kTmDP + c * 16, pd);
+          if (hf == 1) {
+            if (!C::kSep) {
+              // both warpgroups have read their S^T / dP^T columns before either
+              // writes P^T / dS^T over the first half of them
+              okw = named_bar_and(1, 256, okw);
+            } else if (okw && i + 1 < nq) {
+              tc_fence_before();
+              warp_arrive(s_read, lane);
+            }
+          }
+          if (okw) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              float pr[2], dr[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int q = 32 * hf + c + h;
+                const bool v = 64 * e + q < valid_q;
+                const float pv = ex2_approx(fmaf(__uint_as_float(rs[c + h]), sl2, -lse_s[q]));
+                pr[h] = v ? pv : 0.f;
+                dr[h] = v ? pv * (__uint_as_float(rd[c + h]) - dd_s[q]) : 0.f;
+              }
+              pp[hf][c / 2] = pack_bf16(pr[0], pr[1]);
+              pd[hf][c / 2] = pack_bf16(dr[0], dr[1]);
+            }
+          }
         }
+        if (!okw) { ok = false; break; }
+        if (C::kSep && gchunk > 0) {
+          // the dV / dK MMAs of the previous chunk have read P^T / dS^T
+          bool okf = mbar_wait(pd_free, f_waits & 1, ctl, kErrBwdWait);
+          ++f_waits;
+          okf = __all_sync(0xffffffffu, okf);
+          if (!okf) { ok = false; break; }
+          tc_fence_after();
+        }
+        const uint32_t pbase = tmem + lane_off + 32 * e;
+        tmem_st16(pbase + C::kTmP, pp[0]);
+        tmem_st16(pbase + C::kTmP + 16, pp[1]);
+        tmem_st16(pbase + C::kTmDS, pd[0]);
+        tmem_st16(pbase + C::kTmDS + 16, pd[1]);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(p_ready, lane);
         ++ld;
       }
       if (!ok) break;
-      // epilogue: dV, scale * dK -> bf16 rows of this key block
+      // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK (rows of this key block)
       bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
       oke = __all_sync(0xffffffffu, oke);
+      if (!C::kSep) oke = named_bar_and(1, 256, oke);
       if (!oke) { ok = false; break; }
       tc_fence_after();
       const long long tok = row_valid ? token_row(g, p.tiled, bh, ktile, krow) : 0;
+      const uint32_t col = e ? C::kTmDK : C::kTmDV;
+      const float mul = e ? p.scale : 1.f;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(e ? p.dk : p.dv) + tok * D);
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which ? C::kTmDK : C::kTmDV;
-        const float mul = which ? p.scale : 1.f;
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(which ? p.dk : p.dv) + tok * D);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + col + c * 32, r);
+        tmem_ld_wait();
+        if (row_valid) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + col + c * 32, r);
-          tmem_ld_wait();
-          if (row_valid) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
-              w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
-              w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
-              w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
-              dst[c * 4 + v] = w;
-            }
+          for (int v = 0; v < 4; ++v) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
+            w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
+            w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
+            w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
+            dst[c * 4 + v] = w;
           }
         }
       }
@@ -343,14 +417,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------- 3. dQ
+// Warps 0-7 elementwise (warpgroup e = key columns [64 e, 64 e + 64) of each
+// 128-key chunk; thread = query row), warp 8 producer, warp 9 MMA.  dS has
+// TMEM columns of its own, so S / dP of chunk j + 1 are computed while the
+// elementwise warps work on chunk j.
 template <int D>
 struct DqCfg {
   static constexpr uint32_t kTile = kBM * D * 2;
   static constexpr uint32_t kPanel = kBM * 128;
   static constexpr int kSlots = D == 128 ? 4 : 8;
-  static constexpr int kNumBars = 2 * kSlots + 7;
+  // barriers: full[S] empty[S] q_full q_free s_full s_read ds_ready ds_free acc_done acc_free drain
+  static constexpr int kNumBars = 2 * kSlots + 9;
   static constexpr uint32_t kSmem = (2 + kSlots) * kTile + kNumBars * 8 + 64 + 16 + kMaxCoords * 16 + 1024;
-  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDQ = 256;
+  static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDS = 256, kTmDQ = 320;
+  static_assert(kTmDQ + D <= 512, "TMEM budget");
 };
 
 template <int D>
@@ -364,8 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *q_s = smem, *do_s = smem + C::kTile, *slots = smem + 2 * C::kTile;
   uint64_t *bars = reinterpret_cast<uint64_t *>(slots + C::kSlots * C::kTile);
   uint64_t *full = bars, *empty = bars + C::kSlots;
-  uint64_t *q_full = bars + 2 * C::kSlots, *q_free = q_full + 1, *s_full = q_full + 2, *ds_ready = q_full + 3;
-  uint64_t *acc_done = q_full + 4, *acc_free = q_full + 5, *drain = q_full + 6;
+  uint64_t *q_full = bars + 2 * C::kSlots, *q_free = q_full + 1;
+  uint64_t *s_full = q_full + 2;    // S, dP of a chunk are in TMEM
+  uint64_t *s_read = q_full + 3;    // ... and have been read
+  uint64_t *ds_ready = q_full + 4;  // dS written
+  uint64_t *ds_free = q_full + 5;   // the dQ MMAs have read it
+  uint64_t *acc_done = q_full + 6, *acc_free = q_full + 7, *drain = q_full + 8;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int4 *s_coord = reinterpret_cast<int4 *>((reinterpret_cast<uintptr_t>(tmem_slot) + 64 + 15) & ~uintptr_t(15));
@@ -380,9 +464,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
     mbar_init(s_full, 1);
-    mbar_init(ds_ready, 4);
+    mbar_init(s_read, kMathWarps);
+    mbar_init(ds_ready, kMathWarps);
+    mbar_init(ds_free, 1);
     mbar_init(acc_done, 1);
-    mbar_init(acc_free, 4);
+    mbar_init(acc_free, kMathWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -474,42 +560,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qd = smem_desc_sw128(smem_u32(q_s), 16, 1024), dod = smem_desc_sw128(smem_u32(do_s), 16, 1024);
       const uint64_t sk0 = smem_desc_sw128(smem_u32(slots), 16, 1024);         // K-major K / V
       const uint64_t sm0 = smem_desc_sw128(smem_u32(slots), C::kPanel, 1024);  // MN-major K
-      uint32_t ld = 0, item_ctr = 0, ds_waits = 0;
+      uint32_t ld = 0, item_ctr = 0, ds_waits = 0, r_waits = 0;
       bool ok = true, issued = false;
+      // S = Q K^T and dP = dO V^T for chunk j (ring loads lk = K_j, lk + 1 = V_j)
+      auto issue_s = [&](uint32_t lk) -> bool {
+        const uint32_t lv = lk + 1, ks = lk % C::kSlots, vs = lv % C::kSlots;
+        if (!mbar_wait(&full[ks], (lk / C::kSlots) & 1, ctl, kErrBwdWait) ||
+            !mbar_wait(&full[vs], (lv / C::kSlots) & 1, ctl, kErrBwdWait))
+          return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::kTmS, qd + off, sk0 + ((ks * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::kTmDP, dod + off, sk0 + ((vs * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+        mma_commit(&empty[vs]);  // V is read by dP only
+        return true;
+      };
       for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
         const Item it = item_info(item);
         if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
         tc_fence_after();
+        if (!issue_s(ld)) { ok = false; break; }
+        issued = true;
+        if (it.nc == 1) mma_commit(q_free);
         for (int j = 0; j < it.nc && ok; ++j) {
-          const uint32_t lk = ld + 2 * j, lv = lk + 1;
-          const uint32_t ks = lk % C::kSlots, vs = lv % C::kSlots;
-          if (!mbar_wait(&full[ks], (lk / C::kSlots) & 1, ctl, kErrBwdWait) ||
-              !mbar_wait(&full[vs], (lv / C::kSlots) & 1, ctl, kErrBwdWait)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + C::kTmS, qd + off, sk0 + ((ks * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+          const uint32_t lk = ld + 2 * j;
+          if (j + 1 < it.nc) {
+            // the next chunk's S / dP as soon as this chunk's have been read
+            if (!mbar_wait(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+            ++r_waits;
+            tc_fence_after();
+            if (!issue_s(lk + 2)) { ok = false; break; }
+            if (j + 2 == it.nc) mma_commit(q_free);  // Q and dO are no longer read
           }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-            mma_ss(tmem + C::kTmDP, dod + off, sk0 + ((vs * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
-          }
-          issued = true;
-          mma_commit(s_full);
-          mma_commit(&empty[vs]);
-          if (j == it.nc - 1) mma_commit(q_free);
           if (!mbar_wait(ds_ready, ds_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
           ++ds_waits;
           if (j == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
           tc_fence_after();
           // dQ += dS K (keys are the contraction)
+          const uint32_t ks = lk % C::kSlots;
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk)
-            mma_ts(tmem + C::kTmDQ, tmem + C::kTmS + kk * 8, sm0 + ((ks * C::kTile + kk * 16 * 128) >> 4), idesc_dq,
+            mma_ts(tmem + C::kTmDQ, tmem + C::kTmDS + kk * 8, sm0 + ((ks * C::kTile + kk * 16 * 128) >> 4), idesc_dq,
                    (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[ks]);
+          mma_commit(ds_free);
         }
         if (!ok) break;
         ld += 2 * it.nc;
@@ -522,10 +624,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int row = warp * 32 + lane;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    // elementwise warps: thread = query row = TMEM lane; warpgroup e owns key
+    // columns [64 e, 64 e + 64)
+    const int e = warp >> 2, quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const float sl2 = p.scale_log2;
-    uint32_t s_waits = 0, item_ctr = 0;
+    uint32_t s_waits = 0, f_waits = 0, item_ctr = 0, gchunk = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
       const Item it = item_info(item);
@@ -533,33 +638,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_valid = qrow < g.tau;
       const long long lo = it.bh * lse_pitch(g) + (long long)it.tile * g.tau + qrow;
       const float lse2 = row_valid ? p.lse2_t[lo] : 0.f, dd = row_valid ? p.dd_t[lo] : 0.f;
-      for (int j = 0; j < it.nc; ++j) {
+      for (int j = 0; j < it.nc; ++j, ++gchunk) {
         bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
-        const int kvalid = it.nkeys - j * kBM;
-#pragma unroll
-        for (int c = 0; c < kBM / 32; ++c) {
-          uint32_t rs[32], rd[32];
-          tmem_ld32(tmem + lane_off + C::kTmS + c * 32, rs);
-          tmem_ld32(tmem + lane_off + C::kTmDP + c * 32, rd);
-          tmem_ld_wait();
-          uint32_t pd[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float dr[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const bool v = c * 32 + e + h < kvalid;
-              const float pv = ex2_approx(fmaf(__uint_as_float(rs[e + h]), sl2, -lse2));
-              dr[h] = v ? pv * (__uint_as_float(rd[e + h]) - dd) : 0.f;
-            }
-            pd[e / 2] = pack_bf16(dr[0], dr[1]);
-          }
-          tmem_st16(tmem + lane_off + C::kTmS + c * 16, pd);
+        uint32_t rs[2][32], rd[2][32];
+        const uint32_t base = tmem + lane_off + 64 * e;
+        tmem_ld32(base + C::kTmS, rs[0]);
+        tmem_ld32(base + C::kTmS + 32, rs[1]);
+        tmem_ld32(base + C::kTmDP, rd[0]);
+        tmem_ld32(base + C::kTmDP + 32, rd[1]);
+        tmem_ld_wait();
+        if (j + 1 < it.nc) {
+          tc_fence_before();
+          warp_arrive(s_read, lane);
         }
+        const int kvalid = it.nkeys - j * kBM - 64 * e;
+        uint32_t pd[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float dr[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = c + h;
+            const bool v = q < kvalid;
+            const float pv = ex2_approx(fmaf(__uint_as_float(rs[q >> 5][q & 31]), sl2, -lse2));
+            dr[h] = v ? pv * (__uint_as_float(rd[q >> 5][q & 31]) - dd) : 0.f;
+          }
+          pd[c / 2] = pack_bf16(dr[0], dr[1]);
+        }
+        if (gchunk > 0) {
+          // the dQ MMAs of the previous chunk have read dS
+          bool okf = mbar_wait(ds_free, f_waits & 1, ctl, kErrBwdWait);
+          ++f_waits;
+          okf = __all_sync(0xffffffffu, okf);
+          if (!okf) { ok = false; break; }
+          tc_fence_after();
+        }
+        tmem_st32(tmem + lane_off + C::kTmDS + 32 * e, pd);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(ds_ready, lane);
@@ -569,13 +687,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       oke = __all_sync(0xffffffffu, oke);
       if (!oke) { ok = false; break; }
       tc_fence_after();
+      // warpgroup e writes dQ columns [e D / 2, (e + 1) D / 2)
       const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, qrow) : 0;
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dq) + tok * D);
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dq) + tok * D + e * (D / 2));
       const float mul = p.scale;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kTmDQ + c * 32, r);
+        tmem_ld32(tmem + lane_off + C::kTmDQ + e * (D / 2) + c * 32, r);
         tmem_ld_wait();
         if (row_valid) {
 #pragma unroll
