@@ -80,8 +80,10 @@ size_t fwd_workspace(const sta_plan_s *pl) {
 // tile-major with a pitch of N + 128 floats per (batch, head) slice, then (only
 // when tiles are not readable as boxes of the raster tensors) tile-major
 // copies of Q, K, V and dO.
-size_t lse_pitch_bytes(const sta_plan_s *pl) { return ((size_t)pl->g.N + 128) * 4; }
-size_t bwd_vec_bytes(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * lse_pitch_bytes(pl); }
+// LSE * log2(e) and D, one 128-float run per (batch, head, tile, query block)
+size_t bwd_vec_bytes(const sta_plan_s *pl) {
+  return (size_t)pl->g.B * pl->g.Hh * pl->g.n_tiles * pl->nqb * 128 * 4;
+}
 size_t bwd_workspace(const sta_plan_s *pl) {
   size_t b = kStatusBytes + 2 * bwd_vec_bytes(pl);
   b = (b + 255) & ~size_t(255);

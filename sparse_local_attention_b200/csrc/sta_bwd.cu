@@ -50,18 +50,33 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
                : "memory");
 }
 
-__device__ __forceinline__ long long lse_pitch(const Geometry &g) { return (long long)g.N + 128; }
+// LSE * log2(e) and D are stored per 128-row query block: run of block qb of
+// tile t of slice bh = ((bh * n_tiles + t) * nqb + qb) * 128.  Rows past the
+// tile's end hold LSE = +inf and D = 0, so P = exp2(S - LSE) is 0 there and
+// no mask is needed.
+__device__ __forceinline__ long long vec_run(const BwdParams &p, int bh, int tile, int qb) {
+  return (((long long)bh * p.g.n_tiles + tile) * p.nqb + qb) * kBM;
+}
 
 // ----------------------------------------------------------------------- 1. preprocess
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   const Geometry &g = p.g;
   const int lane = threadIdx.x & 31;
-  const long long nrows = (long long)g.B * g.Hh * g.N;
+  const long long nrows = (long long)g.B * g.Hh * g.n_tiles * p.nqb * kBM;  // padded runs
   const long long warps = (long long)gridDim.x * (blockDim.x / 32);
   for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < nrows; r += warps) {
-    const int bh = (int)(r / g.N), pos = (int)(r - (long long)bh * g.N);
-    const int tile = pos / g.tau, o = pos - tile * g.tau;
+    const long long run = r / kBM;
+    const long long bt = run / p.nqb;  // bh * n_tiles + tile
+    const int o = (int)(run - bt * p.nqb) * kBM + (int)(r - run * kBM);
+    const int bh = (int)(bt / g.n_tiles), tile = (int)(bt - (long long)bh * g.n_tiles);
+    if (o >= g.tau) {
+      if (lane == 0) {
+        p.dd_t[r] = 0.f;
+        p.lse2_t[r] = INFINITY;
+      }
+      continue;
+    }
     const long long tok = token_row(g, p.tiled, bh, tile, o);
     const __nv_bfloat16 *orow = static_cast<const __nv_bfloat16 *>(p.o) + tok * D;
     const __nv_bfloat16 *drow = static_cast<const __nv_bfloat16 *>(p.dout) + tok * D;
@@ -76,9 +91,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
-      const long long dst = bh * lse_pitch(g) + pos;
-      p.dd_t[dst] = acc;
-      p.lse2_t[dst] = p.lse[tok] * kLog2e;
+      p.dd_t[r] = acc;
+      p.lse2_t[r] = p.lse[tok] * kLog2e;
     }
   }
 }
@@ -196,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_box<D>(p, &tmap_q, sb + pc * p.piece_rows * 128, c, &st_full[st]);
             load_box<D>(p, &tmap_do, sb + C::kTile + pc * p.piece_rows * 128, c, &st_full[st]);
           }
-          const long long lo = bh * lse_pitch(g) + (long long)qt * g.tau + qb * kBM;
+          const long long lo = vec_run(p, bh, qt, qb);
           bulk_load(sb + 2 * C::kTile, p.lse2_t + lo, 512, &st_full[st]);
           bulk_load(sb + 2 * C::kTile + 512, p.dd_t + lo, 512, &st_full[st]);
           ++ld;
@@ -307,27 +321,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int krow = kb * kBM + row;
       const bool row_valid = krow < g.tau;
       for (int i = 0; i < nq; ++i, ++gchunk) {
-        const int qb = i % p.nqb;
-        const int valid_q = min(kBM, g.tau - qb * kBM);
         const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
         bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
-        // two halves of 32 columns: load, then turn into packed P^T / dS^T
-        const float *lse_s = reinterpret_cast<const float *>(stages + st * C::kStage + 2 * C::kTile) + 64 * e;
-        const float *dd_s = lse_s + 128;
+        // four quarters of 16 columns: load, then turn into packed P^T / dS^T
+        // (query rows past the tile's end have LSE = +inf: P = dS = 0 there)
+        const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + 16 * e;
+        const float4 *dd4 = lse4 + 32;
         uint32_t pp[2][16], pd[2][16];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t rs[32], rd[32];
+        for (int qt = 0; qt < 4; ++qt) {
+          uint32_t rs[16], rd[16];
           if (okw) {
-            if (hf == 0) tc_fence_after();
-            const uint32_t base = tmem + lane_off + 64 * e + 32 * hf;
-            tmem_ld32(base + C::kTmS, rs);
-            tmem_ld32(base + C::kTmDP, rd);
+            if (qt == 0) tc_fence_after();
+            const uint32_t base = tmem + lane_off + 64 * e + 16 * qt;
+            tmem_ld16(base + C::kTmS, rs);
+            tmem_ld16(base + C::kTmDP, rd);
             tmem_ld_wait();
           }
-          if (hf == 1) {
+          if (qt == 3) {
             if (!C::kSep) {
               // both warpgroups have read their S^T / dP^T columns before either
               // writes P^T / dS^T over the first half of them
@@ -339,18 +352,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (okw) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              float pr[2], dr[2];
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const float4 l = lse4[4 * qt + v4], dv = dd4[4 * qt + v4];
+              const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
+              float pr[4], dr[4];
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int q = 32 * hf + c + h;
-                const bool v = 64 * e + q < valid_q;
-                const float pv = ex2_approx(fmaf(__uint_as_float(rs[c + h]), sl2, -lse_s[q]));
-                pr[h] = v ? pv : 0.f;
-                dr[h] = v ? pv * (__uint_as_float(rd[c + h]) - dd_s[q]) : 0.f;
+              for (int h = 0; h < 4; ++h) {
+                const int c = 4 * v4 + h;
+                pr[h] = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -ls[h]));
+                dr[h] = pr[h] * (__uint_as_float(rd[c]) - ds[h]);
               }
-              pp[hf][c / 2] = pack_bf16(pr[0], pr[1]);
-              pd[hf][c / 2] = pack_bf16(dr[0], dr[1]);
+              const int w = 8 * (qt & 1) + 2 * v4;
+              pp[qt >> 1][w] = pack_bf16(pr[0], pr[1]);
+              pp[qt >> 1][w + 1] = pack_bf16(pr[2], pr[3]);
+              pd[qt >> 1][w] = pack_bf16(dr[0], dr[1]);
+              pd[qt >> 1][w + 1] = pack_bf16(dr[2], dr[3]);
             }
           }
         }
@@ -636,8 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = item_info(item);
       const int qrow = it.qb * kBM + row;
       const bool row_valid = qrow < g.tau;
-      const long long lo = it.bh * lse_pitch(g) + (long long)it.tile * g.tau + qrow;
-      const float lse2 = row_valid ? p.lse2_t[lo] : 0.f, dd = row_valid ? p.dd_t[lo] : 0.f;
+      const long long lo = vec_run(p, it.bh, it.tile, it.qb) + row;
+      const float lse2 = p.lse2_t[lo], dd = p.dd_t[lo];
       for (int j = 0; j < it.nc; ++j, ++gchunk) {
         bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
