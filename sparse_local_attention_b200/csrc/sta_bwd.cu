@@ -58,6 +58,34 @@ __device__ __forceinline__ long long vec_run(const BwdParams &p, int bh, int til
   return (((long long)bh * p.g.n_tiles + tile) * p.nqb + qb) * kBM;
 }
 
+// The elementwise pass over one thread's 64 columns of S and dP (TMEM lane =
+// row): four quarters of 16 columns, the TMEM load of quarter q + 1 in flight
+// while quarter q is computed.  compute(q, s, dp) gets the quarter's raw fp32
+// bits; after_reads() runs once every load has completed (the columns may then
+// be overwritten).
+template <typename Compute, typename AfterReads>
+__device__ __forceinline__ void quarters_pipelined(uint32_t s_addr, uint32_t dp_addr, Compute &&compute,
+                                                   AfterReads &&after_reads) {
+  uint32_t s0[16], d0[16], s1[16], d1[16];
+  tmem_ld16(s_addr, s0);
+  tmem_ld16(dp_addr, d0);
+  tmem_ld_wait_regs(s0, d0);
+  tmem_ld16(s_addr + 16, s1);
+  tmem_ld16(dp_addr + 16, d1);
+  compute(0, s0, d0);
+  tmem_ld_wait_regs(s1, d1);
+  tmem_ld16(s_addr + 32, s0);
+  tmem_ld16(dp_addr + 32, d0);
+  compute(1, s1, d1);
+  tmem_ld_wait_regs(s0, d0);
+  tmem_ld16(s_addr + 48, s1);
+  tmem_ld16(dp_addr + 48, d1);
+  compute(2, s0, d0);
+  tmem_ld_wait_regs(s1, d1);
+  after_reads();
+  compute(3, s1, d1);
+}
+
 // ----------------------------------------------------------------------- 1. preprocess
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
@@ -325,50 +353,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
-        // four quarters of 16 columns: load, then turn into packed P^T / dS^T
+        // P^T and dS^T for this warpgroup's 64 query columns, packed to bf16
         // (query rows past the tile's end have LSE = +inf: P = dS = 0 there)
         const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + 16 * e;
         const float4 *dd4 = lse4 + 32;
         uint32_t pp[2][16], pd[2][16];
+        if (okw) {
+          tc_fence_after();
+          const uint32_t base = tmem + lane_off + 64 * e;
+          quarters_pipelined(
+              base + C::kTmS, base + C::kTmDP,
+              [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) {
 #pragma unroll
-        for (int qt = 0; qt < 4; ++qt) {
-          uint32_t rs[16], rd[16];
-          if (okw) {
-            if (qt == 0) tc_fence_after();
-            const uint32_t base = tmem + lane_off + 64 * e + 16 * qt;
-            tmem_ld16(base + C::kTmS, rs);
-            tmem_ld16(base + C::kTmDP, rd);
-            tmem_ld_wait();
-          }
-          if (qt == 3) {
-            if (!C::kSep) {
-              // both warpgroups have read their S^T / dP^T columns before either
-              // writes P^T / dS^T over the first half of them
-              okw = named_bar_and(1, 256, okw);
-            } else if (okw && i + 1 < nq) {
-              tc_fence_before();
-              warp_arrive(s_read, lane);
-            }
-          }
-          if (okw) {
+                for (int v4 = 0; v4 < 4; ++v4) {
+                  const float4 l = lse4[4 * qt + v4], dv = dd4[4 * qt + v4];
+                  const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
+                  float pr[4], dr[4];
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              const float4 l = lse4[4 * qt + v4], dv = dd4[4 * qt + v4];
-              const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
-              float pr[4], dr[4];
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const int c = 4 * v4 + h;
-                pr[h] = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -ls[h]));
-                dr[h] = pr[h] * (__uint_as_float(rd[c]) - ds[h]);
-              }
-              const int w = 8 * (qt & 1) + 2 * v4;
-              pp[qt >> 1][w] = pack_bf16(pr[0], pr[1]);
-              pp[qt >> 1][w + 1] = pack_bf16(pr[2], pr[3]);
-              pd[qt >> 1][w] = pack_bf16(dr[0], dr[1]);
-              pd[qt >> 1][w + 1] = pack_bf16(dr[2], dr[3]);
-            }
-          }
+                  for (int h = 0; h < 4; ++h) {
+                    const int c = 4 * v4 + h;
+                    pr[h] = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -ls[h]));
+                    dr[h] = pr[h] * (__uint_as_float(rd[c]) - ds[h]);
+                  }
+                  const int w = 8 * (qt & 1) + 2 * v4;
+                  pp[qt >> 1][w] = pack_bf16(pr[0], pr[1]);
+                  pp[qt >> 1][w + 1] = pack_bf16(pr[2], pr[3]);
+                  pd[qt >> 1][w] = pack_bf16(dr[0], dr[1]);
+                  pd[qt >> 1][w + 1] = pack_bf16(dr[2], dr[3]);
+                }
+              },
+              [&]() {
+                if (C::kSep && i + 1 < nq) {
+                  tc_fence_before();
+                  warp_arrive(s_read, lane);
+                }
+              });
+        }
+        if (!C::kSep) {
+          // both warpgroups have read their S^T / dP^T columns before either
+          // writes P^T / dS^T over the first half of them
+          okw = named_bar_and(1, 256, okw);
         }
         if (!okw) { ok = false; break; }
         if (C::kSep && gchunk > 0) {
@@ -660,31 +684,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
-        uint32_t rs[2][32], rd[2][32];
-        const uint32_t base = tmem + lane_off + 64 * e;
-        tmem_ld32(base + C::kTmS, rs[0]);
-        tmem_ld32(base + C::kTmS + 32, rs[1]);
-        tmem_ld32(base + C::kTmDP, rd[0]);
-        tmem_ld32(base + C::kTmDP + 32, rd[1]);
-        tmem_ld_wait();
-        if (j + 1 < it.nc) {
-          tc_fence_before();
-          warp_arrive(s_read, lane);
-        }
+        // dS for this warpgroup's 64 key columns, packed to bf16; keys past the
+        // list's end (only in the last chunk) are masked
         const int kvalid = it.nkeys - j * kBM - 64 * e;
-        uint32_t pd[32];
+        const bool whole = kvalid >= 64;
+        uint32_t pd[2][16];
+        const uint32_t base = tmem + lane_off + 64 * e;
+        quarters_pipelined(
+            base + C::kTmS, base + C::kTmDP,
+            [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) {
+              float dr[16];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float dr[2];
+              for (int c = 0; c < 16; ++c) {
+                const float pv = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -lse2));
+                dr[c] = pv * (__uint_as_float(rd[c]) - dd);
+              }
+              if (!whole) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = c + h;
-            const bool v = q < kvalid;
-            const float pv = ex2_approx(fmaf(__uint_as_float(rs[q >> 5][q & 31]), sl2, -lse2));
-            dr[h] = v ? pv * (__uint_as_float(rd[q >> 5][q & 31]) - dd) : 0.f;
-          }
-          pd[c / 2] = pack_bf16(dr[0], dr[1]);
-        }
+                for (int c = 0; c < 16; ++c)
+                  if (16 * qt + c >= kvalid) dr[c] = 0.f;
+              }
+#pragma unroll
+              for (int c = 0; c < 16; c += 2) pd[qt >> 1][8 * (qt & 1) + c / 2] = pack_bf16(dr[c], dr[c + 1]);
+            },
+            [&]() {
+              if (j + 1 < it.nc) {
+                tc_fence_before();
+                warp_arrive(s_read, lane);
+              }
+            });
         if (gchunk > 0) {
           // the dQ MMAs of the previous chunk have read dS
           bool okf = mbar_wait(ds_free, f_waits & 1, ctl, kErrBwdWait);
@@ -693,7 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!okf) { ok = false; break; }
           tc_fence_after();
         }
-        tmem_st32(tmem + lane_off + C::kTmDS + 32 * e, pd);
+        tmem_st16(tmem + lane_off + C::kTmDS + 32 * e, pd[0]);
+        tmem_st16(tmem + lane_off + C::kTmDS + 32 * e + 16, pd[1]);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(ds_ready, lane);
