@@ -287,6 +287,33 @@ def run_ours(args):
                "kernels_per_step": plan.backward_launches}
         del dout, dq, dk, dv, bws
 
+    # --- permute kernel (raster <-> tile-major, HBM-bound): on the forward path
+    #     only when tiles are not TMA boxes of the raster tensor; measured here
+    #     on Q of the same workload, both directions
+    perm_t = torch.empty_like(q)
+    perm_back = torch.empty_like(q)
+    for _ in range(3):
+        sta.sta_permute(plan, q, perm_t, stream=stream)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    perm_reps = 10
+    p0.record(stream)
+    for _ in range(perm_reps):
+        sta.sta_permute(plan, q, perm_t, stream=stream)
+        sta.sta_permute(plan, perm_t, perm_back, inverse=True, stream=stream)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    perm_ms = p0.elapsed_time(p1) / (2 * perm_reps)
+    if not torch.equal(perm_back, q):
+        raise RuntimeError("permute round trip is not the identity")
+    perm_bytes = 2 * q.numel() * q.element_size()  # read + write
+    hbm_peak = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    permute = {"kernel": "permute_kernel", "ms_per_launch": perm_ms, "bytes_per_launch": perm_bytes,
+               "achieved_gbs": perm_bytes / (perm_ms * 1e-3) / 1e9, "peak_gbs": hbm_peak,
+               "frac": perm_bytes / (perm_ms * 1e-3) / 1e9 / hbm_peak,
+               "peak_source": f"{pk_kind} hbm_gbs", "bound": "hbm"}
+    del perm_t, perm_back
+
     # --- end to end through the public API: pinned host in, host out
     o_h = torch.empty_like(q_h).pin_memory()
     lse_h = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32).pin_memory()
@@ -365,6 +392,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "dense_baseline": dense,
             "backward": bwd,
+            "permute": permute,
         }
         print(json.dumps(out), flush=True)
     plan.destroy()

@@ -7,9 +7,12 @@
 // to position tile*tau + in_tile, tile = ((t/tt)*GH + h/th)*GW + w/tw and
 // in_tile = ((t%tt)*th + h%th)*tw + w%tw.
 //
-// One thread moves 16 bytes (8 bf16).  Threads walk the tile-major side in
-// order, so that side is perfectly coalesced; on the raster side a warp still
-// touches runs of tile_w whole token rows (tile_w * d * 2 contiguous bytes).
+// One CTA per (batch x head slice, tile).  Inside a tile, the tokens of one
+// (t, h) line form a run of tile_w consecutive tokens on both sides (raster
+// and tile-major), so the CTA walks the tile run by run in 16-byte chunks:
+// both sides are read and written in contiguous runs of tile_w * d * 2 bytes,
+// and the only index arithmetic per chunk is two 32-bit divisions.  Each
+// thread keeps four chunks in flight.
 #include <cuda_bf16.h>
 
 #include "sta_kernels.h"
@@ -17,41 +20,57 @@
 namespace sta {
 namespace {
 
-__global__ void __launch_bounds__(256) permute_kernel(const PermuteParams p) {
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) permute_kernel(const PermuteParams p) {
   const Geometry &g = p.g;
-  const int cpr = g.d / 8;  // 16-byte chunks per row
-  const long long total = (long long)g.B * g.Hh * g.N * cpr;
+  const int cpr = g.d / 8;        // 16-byte chunks per token row
+  const int run = g.tw * cpr;     // chunks in one (t, h) line of the tile
+  const int total = g.tt * g.th * run;
   const uint4 *src = static_cast<const uint4 *>(p.src);
   uint4 *dst = static_cast<uint4 *>(p.dst);
-  const int plane = g.th * g.tw;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long row = i / cpr;
-    const int c = (int)(i - row * cpr);
-    const long long bh = row / g.N;
-    const int pos = (int)(row - bh * g.N);  // tile-major position
-    const int tile = pos / g.tau, o = pos - (pos / g.tau) * g.tau;
+  for (long long slab = blockIdx.x; slab < (long long)g.B * g.Hh * g.n_tiles; slab += gridDim.x) {
+    const int bh = (int)(slab / g.n_tiles), tile = (int)(slab - (long long)bh * g.n_tiles);
     const int it = tile / (g.GH * g.GW), ih = (tile / g.GW) % g.GH, iw = tile % g.GW;
-    const int a = o / plane, b = (o / g.tw) % g.th, cc = o % g.tw;
-    const long long n = ((long long)(it * g.tt + a) * g.H + (ih * g.th + b)) * g.W + (iw * g.tw + cc);
-    const long long raster = (bh * g.N + n) * cpr + c;
-    const long long tiled = row * cpr + c;
-    if (p.inverse)
-      dst[raster] = src[tiled];
-    else
-      dst[tiled] = src[raster];
+    const long long tiled0 = ((long long)bh * g.N + (long long)tile * g.tau) * cpr;
+    const long long raster0 = (long long)bh * g.N * cpr;
+    auto offsets = [&](int idx, long long &raster, long long &tiled) {
+      const int r = idx / run, c = idx - r * run;  // line of the tile, chunk in the line
+      const int a = r / g.th, b = r - a * g.th;
+      const long long n = ((long long)(it * g.tt + a) * g.H + (ih * g.th + b)) * g.W + iw * g.tw;
+      raster = raster0 + n * cpr + c;
+      tiled = tiled0 + (long long)r * run + c;
+    };
+    for (int base = threadIdx.x; base < total; base += kThreads * kUnroll) {
+      long long from[kUnroll], to[kUnroll];
+      uint4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int idx = base + u * kThreads;
+        if (idx < total) {
+          long long raster, tiled;
+          offsets(idx, raster, tiled);
+          from[u] = p.inverse ? tiled : raster;
+          to[u] = p.inverse ? raster : tiled;
+          v[u] = src[from[u]];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + u * kThreads < total) dst[to[u]] = v[u];
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_permute(const PermuteParams &p, int num_sms, cudaStream_t stream) {
-  const long long total = (long long)p.g.B * p.g.Hh * p.g.N * (p.g.d / 8);
-  if (total == 0) return cudaSuccess;
-  long long blocks = (total + 255) / 256;
-  const long long cap = (long long)num_sms * 16;
-  if (blocks > cap) blocks = cap;
-  permute_kernel<<<(int)blocks, 256, 0, stream>>>(p);
+  const long long slabs = (long long)p.g.B * p.g.Hh * p.g.n_tiles;
+  if (slabs == 0) return cudaSuccess;
+  const long long cap = (long long)num_sms * 8;  // 8 CTAs of 256 threads per SM
+  const int blocks = (int)(slabs < cap ? slabs : cap);
+  permute_kernel<<<blocks, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -73,6 +73,9 @@ SMALL = {
     "d128_permute_fallback": Workload("e", 1, 2, 128, 4, 12, 8, (2, 6, 4), ((3, 1, 2), (2, 2, 2))),
     "d64_single_tile_grid": Workload("f", 2, 1, 64, 2, 8, 8, (2, 8, 8), ((3, 3, 3),)),
     "d128_tau8_tiny_tiles": Workload("g", 1, 2, 128, 4, 4, 8, (1, 2, 4), ((3, 3, 3), (2, 1, 2))),
+    # 2D (image) STA: a one-frame latent with 1 x th x tw tiles
+    "d64_image_2d": Workload("n", 1, 2, 64, 1, 32, 48, (1, 8, 8), ((1, 3, 3), (1, 5, 5))),
+    "d128_image_2d_tau256": Workload("o", 1, 1, 128, 1, 64, 64, (1, 16, 16), ((1, 3, 3),)),
     # windows that are distinct for some tiles: their last blocks stay lone (split across warpgroups)
     "d128_lone_blocks_split": Workload("l", 1, 2, 128, 4, 8, 32, (2, 8, 8), ((1, 1, 2), (1, 1, 3))),
     "d64_lone_block_odd_chunks": Workload("m", 2, 1, 64, 2, 8, 40, (2, 8, 8), ((1, 1, 3),)),

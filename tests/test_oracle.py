@@ -92,6 +92,7 @@ SMALL_CASES = [
     (4, 6, 8, (2, 2, 2), [(1, 3, 2), (2, 2, 4), (5, 5, 5)]),  # 2x3x4 grid
     (3, 8, 8, (1, 2, 2), [(7, 7, 7), (2, 3, 1), (1, 1, 1)]),  # 3x4x4 grid
     (5, 4, 6, (1, 2, 3), [(2, 1, 2), (4, 2, 1)]),            # 5x2x2 grid, even widths
+    (1, 8, 12, (1, 2, 2), [(1, 3, 3), (1, 2, 5)]),           # 2D (image): one frame, 1x4x6 grid
 ]
 
 
