@@ -132,24 +132,34 @@ def dist_env():
     return world, rank, local
 
 
-def init_dist(world, local):
+def init_dist(world, local, backend="nccl"):
+    """Process group for barriers and max-over-ranks timing only (the ranks
+    share no data).  NCCL on the GPUs; gloo serves the host-side tests."""
     if world > 1:
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
         return dist
     return None
 
 
-def max_over_ranks(dist, x: float) -> float:
+def max_over_ranks(dist, x: float, device="cuda") -> float:
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Throughput of the whole job: the units every rank processed over the
+    slowest rank's time (weak scaling: each rank has its own problem)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -261,7 +271,7 @@ def run_ours(args):
     ms_rank = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(dist, ms_rank)
     flops = wl.forward_flops()
-    value = flops * world / (ms * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, ms) / 1e12
     launches_per_step = plan.forward_launches  # kernels one sta_forward call enqueues
 
     # --- backward (fine-tuning workloads): dQ, dK, dV from the same inputs

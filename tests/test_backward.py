@@ -90,8 +90,9 @@ def test_backward_is_deterministic():
 
 def test_finetune_sampled_rows():
     """The fine-tuning workload (2x16 heads, 16x64x64, tile 4x8x8, window
-    3x5x5): dQ on sampled rows of 64 query tiles for 4 slices, dK/dV on rows of
-    8 key tiles (4 corners + 4 seeded) for 2 slices."""
+    3x5x5): dQ on sampled rows of 64 query tiles for 4 slices, dK/dV on
+    sampled rows of 64 key tiles (8 corners + 56 seeded) for the same 4
+    slices."""
     wl = WORKLOADS["finetune"]
     q, k, v, do = make_inputs(wl, with_dout=True)
     _, _, (dq, dk, dv) = run_fwd_bwd(wl, q, k, v, do)
@@ -108,10 +109,8 @@ def test_finetune_sampled_rows():
         b, h = divmod(bh, wl.Hh)
         rdq, _, _ = oracle.backward(g, q, k, v, do, bh, q_rows=rows, k_rows=np.zeros(0, dtype=np.int64))
         compare(f"dq[{bh}]", dq[b, h, torch.as_tensor(rows)].double().cpu().numpy(), rdq)
-    gt, gh, gw = wl.grid
-    corners = [0, gw - 1, (gh - 1) * gw, gt * gh * gw - 1]
-    for bh in slices[:2]:
-        ktiles = corners + [int(x) for x in rng.choice(wl.n_tiles, 4, replace=False)]
+    ktiles = tiles_sample(wl, 64, seed=1)
+    for bh in slices:
         rows = []
         for t in ktiles:
             toks = tile_tokens(wl, t)

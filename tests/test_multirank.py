@@ -1,0 +1,65 @@
+"""The N > 1 path of bench.py on the host: two gloo ranks on the CPU (no GPU,
+no data-path collective).  Checks max-over-ranks timing, the whole-job rate,
+per-rank seeds and that the reference arm runs on rank 0 only."""
+import contextlib
+import io
+import os
+import socket
+import sys
+
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_local_attention_b200.workloads import WORKLOADS, make_inputs
+
+    w, r, local = bench.dist_env()
+    dist = bench.init_dist(w, local, backend="gloo")
+    try:
+        # each rank times its own problem; the job's time is the slowest rank's
+        ms = bench.max_over_ranks(dist, 10.0 + 5.0 * rank, device="cpu")
+        rate = bench.whole_job_rate(1e12, w, ms)
+        # ranks draw different inputs (independent problems)
+        q = make_inputs(WORKLOADS["tiny"], seed=r)[0]
+        first = torch.tensor([float(q.float().sum())])
+        gathered = [torch.zeros(1) for _ in range(w)]
+        dist.all_gather(gathered, first)
+        # the reference arm: rank 0 only, the others return 0 without output
+        out = io.StringIO()
+        if r != 0:
+            with contextlib.redirect_stdout(out):
+                code = bench.run_reference(None)
+        else:
+            code = 0
+        dist.barrier()
+        results[rank] = (w, r, ms, rate, [float(x) for x in gathered], code, out.getvalue())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_worker, args=(world, _free_port(), results), nprocs=world, start_method="spawn", join=True)
+    assert sorted(results.keys()) == [0, 1]
+    for rank in range(world):
+        w, r, ms, rate, gathered, code, out = results[rank]
+        assert (w, r) == (world, rank)
+        assert ms == 15.0                       # max over ranks, same on every rank
+        assert rate == 1e12 * world / 15e-3     # all ranks' units over the slowest time
+        assert gathered[0] != gathered[1]       # per-rank seeds
+        assert code == 0 and out == ""
