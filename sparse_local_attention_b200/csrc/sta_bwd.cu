@@ -354,42 +354,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
         // P^T and dS^T for this warpgroup's 64 query columns, packed to bf16
-        // (query rows past the tile's end have LSE = +inf: P = dS = 0 there)
+        // (query rows past the tile's end have LSE = +inf: P = dS = 0 there).
         const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + 16 * e;
         const float4 *dd4 = lse4 + 32;
         uint32_t pp[2][16], pd[2][16];
-        if (okw) {
-          tc_fence_after();
-          const uint32_t base = tmem + lane_off + 64 * e;
-          quarters_pipelined(
-              base + C::kTmS, base + C::kTmDP,
-              [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) {
+        // columns q0 .. q0 + 4 n - 1 of P^T / dS^T from raw S^T / dP^T bits
+        auto pds = [&](int q0, int n, const uint32_t *rs, const uint32_t *rd) {
 #pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
-                  const float4 l = lse4[4 * qt + v4], dv = dd4[4 * qt + v4];
-                  const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
-                  float pr[4], dr[4];
+          for (int v4 = 0; v4 < n; ++v4) {
+            const float4 l = lse4[q0 / 4 + v4], dv = dd4[q0 / 4 + v4];
+            const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
+            float pr[4], dr[4];
 #pragma unroll
-                  for (int h = 0; h < 4; ++h) {
-                    const int c = 4 * v4 + h;
-                    pr[h] = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -ls[h]));
-                    dr[h] = pr[h] * (__uint_as_float(rd[c]) - ds[h]);
-                  }
-                  const int w = 8 * (qt & 1) + 2 * v4;
-                  pp[qt >> 1][w] = pack_bf16(pr[0], pr[1]);
-                  pp[qt >> 1][w + 1] = pack_bf16(pr[2], pr[3]);
-                  pd[qt >> 1][w] = pack_bf16(dr[0], dr[1]);
-                  pd[qt >> 1][w + 1] = pack_bf16(dr[2], dr[3]);
-                }
-              },
-              [&]() {
-                if (C::kSep && i + 1 < nq) {
-                  tc_fence_before();
-                  warp_arrive(s_read, lane);
-                }
-              });
-        }
-        if (!C::kSep) {
+            for (int h = 0; h < 4; ++h) {
+              pr[h] = ex2_approx(fmaf(__uint_as_float(rs[4 * v4 + h]), sl2, -ls[h]));
+              dr[h] = pr[h] * (__uint_as_float(rd[4 * v4 + h]) - ds[h]);
+            }
+            const int w = (q0 + 4 * v4) / 2;  // packed column of the warpgroup's 32
+            pp[w >> 4][w & 15] = pack_bf16(pr[0], pr[1]);
+            pp[w >> 4][(w & 15) + 1] = pack_bf16(pr[2], pr[3]);
+            pd[w >> 4][w & 15] = pack_bf16(dr[0], dr[1]);
+            pd[w >> 4][(w & 15) + 1] = pack_bf16(dr[2], dr[3]);
+          }
+        };
+        if constexpr (C::kSep) {
+          // S^T and dP^T are read in one batch and their columns released at
+          // once: the MMA warp computes the next chunk's while this one is done
+          uint32_t rs[2][32], rd[2][32];
+          if (okw) {
+            tc_fence_after();
+            const uint32_t base = tmem + lane_off + 64 * e;
+            tmem_ld32(base + C::kTmS, rs[0]);
+            tmem_ld32(base + C::kTmS + 32, rs[1]);
+            tmem_ld32(base + C::kTmDP, rd[0]);
+            tmem_ld32(base + C::kTmDP + 32, rd[1]);
+            tmem_ld_wait();
+            if (i + 1 < nq) {
+              tc_fence_before();
+              warp_arrive(s_read, lane);
+            }
+            pds(0, 8, rs[0], rd[0]);
+            pds(32, 8, rs[1], rd[1]);
+          }
+        } else {
+          // P^T / dS^T are written over S^T / dP^T, so their columns are not
+          // released early: four quarters, the next quarter's load in flight
+          if (okw) {
+            tc_fence_after();
+            const uint32_t base = tmem + lane_off + 64 * e;
+            quarters_pipelined(
+                base + C::kTmS, base + C::kTmDP,
+                [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) { pds(16 * qt, 4, rs, rd); },
+                [&]() {});
+          }
           // both warpgroups have read their S^T / dP^T columns before either
           // writes P^T / dS^T over the first half of them
           okw = named_bar_and(1, 256, okw);
@@ -684,35 +701,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
-        // dS for this warpgroup's 64 key columns, packed to bf16; keys past the
-        // list's end (only in the last chunk) are masked
+        // dS for this warpgroup's 64 key columns, packed to bf16.  S and dP are
+        // read in one batch so the MMA warp can reuse their columns at once;
+        // keys past the list's end (only in the last chunk) are masked.
         const int kvalid = it.nkeys - j * kBM - 64 * e;
         const bool whole = kvalid >= 64;
-        uint32_t pd[2][16];
+        uint32_t rs[2][32], rd[2][32];
         const uint32_t base = tmem + lane_off + 64 * e;
-        quarters_pipelined(
-            base + C::kTmS, base + C::kTmDP,
-            [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) {
-              float dr[16];
+        tmem_ld32(base + C::kTmS, rs[0]);
+        tmem_ld32(base + C::kTmS + 32, rs[1]);
+        tmem_ld32(base + C::kTmDP, rd[0]);
+        tmem_ld32(base + C::kTmDP + 32, rd[1]);
+        tmem_ld_wait();
+        if (j + 1 < it.nc) {
+          tc_fence_before();
+          warp_arrive(s_read, lane);
+        }
+        uint32_t pd[2][16];
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const float pv = ex2_approx(fmaf(__uint_as_float(rs[c]), sl2, -lse2));
-                dr[c] = pv * (__uint_as_float(rd[c]) - dd);
-              }
-              if (!whole) {
+        for (int hf = 0; hf < 2; ++hf) {
+          float dr[32];
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                  if (16 * qt + c >= kvalid) dr[c] = 0.f;
-              }
+          for (int c = 0; c < 32; ++c) {
+            const float pv = ex2_approx(fmaf(__uint_as_float(rs[hf][c]), sl2, -lse2));
+            dr[c] = pv * (__uint_as_float(rd[hf][c]) - dd);
+          }
+          if (!whole) {
 #pragma unroll
-              for (int c = 0; c < 16; c += 2) pd[qt >> 1][8 * (qt & 1) + c / 2] = pack_bf16(dr[c], dr[c + 1]);
-            },
-            [&]() {
-              if (j + 1 < it.nc) {
-                tc_fence_before();
-                warp_arrive(s_read, lane);
-              }
-            });
+            for (int c = 0; c < 32; ++c)
+              if (32 * hf + c >= kvalid) dr[c] = 0.f;
+          }
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) pd[hf][c / 2] = pack_bf16(dr[c], dr[c + 1]);
+        }
         if (gchunk > 0) {
           // the dQ MMAs of the previous chunk have read dS
           bool okf = mbar_wait(ds_free, f_waits & 1, ctl, kErrBwdWait);
