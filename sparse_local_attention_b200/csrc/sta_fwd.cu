@@ -62,8 +62,8 @@ struct FwdCfg {
   static constexpr int kSlots = (D == 128 ? 4 : 8) + (2 - kNumQ);
   static constexpr uint32_t kTmO0 = 256;  // O_X at kTmO0 + X * D; S_X at 128 * X
   static constexpr uint32_t kTmCols = 512;
-  // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain
-  static constexpr int kNumBars = 2 * kSlots + 11;
+  // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain p_half[2]
+  static constexpr int kNumBars = 2 * kSlots + 13;
   static constexpr uint32_t kMiscBytes = 64 + 4 * 128 * 4;  // tmem address, abort flag, m/l exchange
   static constexpr uint32_t kListBytes = kMaxCoords * 16;
   static constexpr uint32_t kSmemBytes =
@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *pv_done = p_ready + 2;          // [2]
   uint64_t *o_free = pv_done + 2;           // [2]
   uint64_t *drain = o_free + 2;
+  uint64_t *p_half = drain + 1;             // [2] P of the chunk's first 64 keys written
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *ml_xchg = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(tmem_slot) + 64);  // [m0 m1 l0 l1][128]
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
       mbar_init(&p_ready[x], 4);  // the four warps of the block's warpgroup
+      mbar_init(&p_half[x], 4);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_free[x], 4);
     }
@@ -281,14 +283,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&s_full[x]);
       };
-      // O_X += P_X V for the V chunk in ring slot `slot`.
-      auto mma_pv = [&](int x, uint32_t slot, bool first) {
+      // O_X += P_X V for the V chunk in ring slot `slot`, in two halves of 64
+      // keys: the first is issued as soon as the softmax has written P for
+      // those keys, the second (and the pv_done commit) once all of P is there.
+      auto mma_pv = [&](int x, uint32_t slot, bool first, uint32_t ph) -> bool {
         const uint64_t vd = vdesc0 + ((slot * C::kTileBytes) >> 4);
         const uint32_t o_tm = tmem + C::kTmO0 + x * D, p_tm = tmem + 128 * x;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int kk = 0; kk < kBN / 32; ++kk)
           mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        if (!mbar_wait(&p_ready[x], ph, ctl, kErrWaitMma)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+          mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, 1u);
         mma_commit(&pv_done[x]);
+        return true;
       };
       auto wait_slot = [&](uint32_t slot_ld) -> bool {
         const uint32_t slot = slot_ld % C::kSlots, phase = (slot_ld / C::kSlots) & 1;
@@ -313,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < it.nc && ok; ++j) {
             const uint32_t vj = k0 + 2 * j + 1, kn = k0 + 2 * j + 2;  // V_j, K_{j+1} load indices
             for (int x = 0; x < nx; ++x) {
-              if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+              const uint32_t ph = p_waits[x] & 1;
+              if (!mbar_wait(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
               }
               if (x == 0 && !wait_slot(vj)) { ok = false; break; }
-              mma_pv(x, vj % C::kSlots, j == 0);
+              if (!mma_pv(x, vj % C::kSlots, j == 0, ph)) { ok = false; break; }
               if (x == nx - 1) mma_commit(&empty[vj % C::kSlots]);
               if (j + 1 < it.nc) {
                 if (x == 0 && !wait_slot(kn)) { ok = false; break; }
@@ -368,7 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < it.n(0) && ok; ++j) {
             for (int x = 0; x < nx; ++x) {
               if (j >= it.n(x)) continue;
-              if (!mbar_wait(&p_ready[x], p_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+              const uint32_t ph = p_waits[x] & 1;
+              if (!mbar_wait(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
@@ -378,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
               }
               if (!take(vslot)) { ok = false; break; }
-              mma_pv(x, vslot % C::kSlots, j == 0);
+              if (!mma_pv(x, vslot % C::kSlots, j == 0, ph)) { ok = false; break; }
               release(vslot);
               if (j + 1 < it.n(x)) {
                 if (!take(kslot)) { ok = false; break; }
@@ -470,7 +482,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool warp_resc = __any_sync(0xffffffffu, resc) && j > 0;
         m = m_new;
 
-        // P = exp2(S * scale_log2 - m) as bf16 over the consumed S columns, row sum
+        // P = exp2(S * scale_log2 - m) as bf16 over the consumed S columns, row
+        // sum.  The first 64 keys are published on their own (p_half) so that
+        // half of P V runs while the rest of P is formed; O is rescaled (rarely)
+        // before that, once the first half of S is no longer held.
         float ls[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) ls[a] = 0.f;
@@ -485,19 +500,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[i / 2] = pack_bf16(p0, p1);
           }
           tmem_st16(tmem + lane_off + s_col + c * 16, pk);
-        }
-        l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
-        if (warp_resc) {
+          if (c == 1) {
+            if (warp_resc) {
+              // O holds every chunk before j (P V(j-1) finished before S(j))
+#pragma unroll 1
+              for (int oc = 0; oc < D / 16; ++oc) {
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_off + o_col + oc * 16, r);
+                tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_off + o_col + c * 32, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tmem + lane_off + o_col + c * 32, r);
+                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                tmem_st16(tmem + lane_off + o_col + oc * 16, r);
+              }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            warp_arrive(&p_half[x], lane);
           }
         }
+        l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(&p_ready[x], lane);
