@@ -374,24 +374,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA and integer pipes, for x <= 8: x = n + f with n = round(x)
-// and f in [-1/2, 1/2]; 2^f from a cubic whose coefficients were fitted here
-// to 2^f on [-1/2, 1/2] by relative-error-weighted least squares iterated
-// towards minimax (max relative error 7.5e-5 in fp32, far below bf16's
-// rounding step); 2^n is added to the exponent field.  Inputs below -126 are
-// clamped there (result ~1e-38, which is what a masked score contributes).
-// The round-to-nearest uses the 1.5 * 2^23 shifter: the integer lands in the
-// low mantissa bits of t, and (bits(t) << 23) is exactly n << 23 because the
-// shifter's own low nine bits are zero.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float q = fmaf(fmaf(fmaf(0.05517090484499931f, f, 0.24260953068733215f), f, 0.6932609677314758f), f,
-                       0.9999281764030457f);
-  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
-}
-
 // Three-input maximum (sm_100).
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -419,15 +401,6 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
       : "r"((uint32_t)v), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
-}
-
-// Pack two non-negative fp32 values into bf16x2, rounding to nearest with
-// ties away from zero, on the integer pipe (lo -> bits 0..15).  Used for the
-// softmax probabilities so the conversion does not compete with ex2 for the
-// XU pipe; it differs from round-to-nearest-even only on exact ties.
-__device__ __forceinline__ uint32_t pack_bf16_rna(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
