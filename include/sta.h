@@ -152,6 +152,28 @@ sta_status sta_forward(sta_plan_t plan, const void *q, const void *k, const void
                        float *lse, void *workspace, size_t workspace_bytes, void *stream,
                        uint32_t flags);
 
+/* Device workspace that sta_forward_host needs: device copies of q, k, v, o
+ * and lse, then sta_forward's own workspace.  This call has no counterpart in
+ * the paper. */
+sta_status sta_plan_host_workspace_size(sta_plan_t plan, size_t *bytes);
+
+/* Forward pass on HOST tensors (same computation and layouts as sta_forward):
+ * q, k, v are read from host memory and o (and lse, nullable) written to host
+ * memory; `workspace` is device memory of at least
+ * sta_plan_host_workspace_size bytes, 16-byte aligned.  The (batch, head)
+ * slices are processed in up to 8 groups: the inputs of one group are copied
+ * to the device while the previous group is computed, and each group's
+ * outputs are copied back while later groups run, on two internal streams
+ * ordered against `stream` with events (one cudaMemcpyAsync per tensor and
+ * group).  The call returns after enqueueing; when `stream` reaches the end of
+ * the call, o and lse are in host memory.  Copies overlap only for page-locked
+ * host memory.  With tiles that are not TMA boxes of the raster tensor, or
+ * with STA_PROBLEM_CTA_PAIR, the whole tensors are copied in, computed and
+ * copied out in order.  Host buffers must stay valid and unchanged until
+ * `stream` has passed the call.  This call has no counterpart in the paper. */
+sta_status sta_forward_host(sta_plan_t plan, const void *q, const void *k, const void *v, void *o, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream, uint32_t flags);
+
 /* Backward pass for the fine-tuning case ("Fast Video Generation with Sliding
  * Tile Attention", Abstract: fine-tuning with STA).  With P = softmax of the
  * windowed scores and D_i = sum_c dO_ic O_ic:

@@ -31,6 +31,10 @@ struct sta_plan_s {
   std::vector<int32_t> inv_off;  // [heads][n_tiles + 1], absolute into inv_idx
   std::vector<int32_t> inv_idx;
   std::vector<int4> work;        // forward work items (see FwdParams::work)
+  // sta_forward_host: the same items grouped by slice group (slices
+  // [group_slice[g], group_slice[g + 1])), two-block items then lone ones
+  std::vector<int4> work_host;
+  std::vector<int> group_off, group_lone, group_slice;
   std::vector<int2> work_kv;     // backward dK/dV items (bh, key tile * nqb + key block)
   std::vector<int2> work_q;      // backward dQ items (bh, query tile * nqb + query block)
   int nqb = 1;  // 128-row query blocks per tile
@@ -45,7 +49,7 @@ struct sta_plan_s {
   int device = -1, num_sms = 0;
   // device copies
   int32_t *d_kv_list = nullptr, *d_count = nullptr, *d_inv_off = nullptr, *d_inv_idx = nullptr;
-  int4 *d_work = nullptr;
+  int4 *d_work = nullptr, *d_work_host = nullptr;
   int2 *d_work_kv = nullptr, *d_work_q = nullptr;
 };
 
@@ -76,14 +80,25 @@ size_t fwd_workspace(const sta_plan_s *pl) {
   return b;
 }
 
-// Backward workspace: status word, then LSE*log2(e) and D = rowsum(dO*O),
-// tile-major with a pitch of N + 128 floats per (batch, head) slice, then (only
-// when tiles are not readable as boxes of the raster tensors) tile-major
-// copies of Q, K, V and dO.
-// LSE * log2(e) and D, one 128-float run per (batch, head, tile, query block)
+// Backward workspace: status word, then LSE*log2(e) and D = rowsum(dO*O), one
+// 128-float run per (batch, head, tile, query block), then (only when tiles
+// are not readable as boxes of the raster tensors) tile-major copies of Q, K, V
+// and dO.
 size_t bwd_vec_bytes(const sta_plan_s *pl) {
   return (size_t)pl->g.B * pl->g.Hh * pl->g.n_tiles * pl->nqb * 128 * 4;
 }
+// sta_forward_host workspace: device copies of Q, K, V, O and LSE (each at a
+// 256-byte boundary), then sta_forward's own workspace (status word first).
+constexpr int kHostGroups = 8;  // slice groups pipelined by sta_forward_host
+
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t lse_bytes(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * pl->g.N * 4; }
+
+size_t host_copies_bytes(const sta_plan_s *pl) { return 4 * round256(tensor_bytes(pl)) + round256(lse_bytes(pl)); }
+
+size_t host_workspace(const sta_plan_s *pl) { return host_copies_bytes(pl) + fwd_workspace(pl); }
+
 size_t bwd_workspace(const sta_plan_s *pl) {
   size_t b = kStatusBytes + 2 * bwd_vec_bytes(pl);
   b = (b + 255) & ~size_t(255);
@@ -163,10 +178,11 @@ void free_device(sta_plan_s *pl) {
   cudaFree(pl->d_inv_off);
   cudaFree(pl->d_inv_idx);
   cudaFree(pl->d_work);
+  cudaFree(pl->d_work_host);
   cudaFree(pl->d_work_kv);
   cudaFree(pl->d_work_q);
   pl->d_kv_list = pl->d_count = pl->d_inv_off = pl->d_inv_idx = nullptr;
-  pl->d_work = nullptr;
+  pl->d_work = pl->d_work_host = nullptr;
   pl->d_work_kv = pl->d_work_q = nullptr;
 }
 
@@ -217,6 +233,52 @@ sta_status finish_call(const sta_plan_s *pl, void *workspace, cudaStream_t strea
   }
   (void)pl;
   return STA_OK;
+}
+
+struct ForwardMaps {
+  CUtensorMap q, k, v, kh, vh;
+  bool ok = false;
+};
+
+// Tensor maps of one forward call over Q, K, V at qbase / kbase / vbase (raster
+// boxes, or tile-major rows when the tensors are tile-major or gathered).
+ForwardMaps forward_maps(const sta_plan_s *pl, const void *qbase, const void *kbase, const void *vbase) {
+  ForwardMaps m;
+  const bool raster5d = pl->kv_mode == sta::kKvRaster;
+  m.ok = raster5d ? (make_map_raster(&m.q, qbase, pl) && make_map_raster(&m.k, kbase, pl) &&
+                     make_map_raster(&m.v, vbase, pl))
+                  : (make_map_tiled(&m.q, qbase, pl) && make_map_tiled(&m.k, kbase, pl) &&
+                     make_map_tiled(&m.v, vbase, pl));
+  if (m.ok && pl->pair)
+    m.ok = raster5d ? (make_map_raster_box(&m.kh, kbase, pl, pl->kh_box[0], pl->kh_box[1], pl->kh_box[2], 2) &&
+                       make_map_raster_box(&m.vh, vbase, pl, pl->vh_box[0], pl->vh_box[1], pl->vh_box[2], 1))
+                    : (make_map_tiled_box(&m.kh, kbase, pl, 64, 2) && make_map_tiled_box(&m.vh, vbase, pl, 128, 1));
+  return m;
+}
+
+// Launch the forward kernel(s) over `n_work` items at `work` (the last
+// `n_lone` of them lone blocks).
+sta_status enqueue_forward(const sta_plan_s *pl, const ForwardMaps &maps, const void *q, void *o, float *lse,
+                           int *status, cudaStream_t stream, const int4 *work, int n_work, int n_lone) {
+  const bool raster5d = pl->kv_mode == sta::kKvRaster;
+  sta::FwdParams fp{};
+  fp.g = pl->g;
+  fp.q = q, fp.o = o, fp.lse = lse;
+  fp.tiled = pl->tiled ? 1 : 0;
+  fp.nqb = pl->nqb;
+  fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
+  fp.work = work, fp.n_work = n_work, fp.n_work_lone = n_lone;
+  fp.scale_log2 = pl->scale * 1.4426950408889634f;
+  fp.status = status;
+  fp.wait_limit_ns = g_wait_limit_ns;
+  fp.kv_mode = raster5d ? sta::kKvRaster : sta::kKvTiled;
+  fp.piece_rows = pl->piece_rows;
+  fp.box_w = pl->box_w, fp.box_h = pl->box_h, fp.box_t = pl->box_t;
+  fp.box_panels = box_panels(pl);
+  fp.oob_coord = raster5d ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
+  const cudaError_t e = pl->pair ? sta::launch_forward_pair(fp, maps.kh, maps.vh, pl->num_sms, stream)
+                                 : sta::launch_forward(fp, maps.q, maps.k, maps.v, pl->num_sms, stream);
+  return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
 }
 
 }  // namespace
@@ -385,6 +447,28 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     std::stable_sort(lone_items.begin(), lone_items.end(), by_cost);
     pl->n_work_lone = (int)lone_items.size();
     pl->work.insert(pl->work.end(), lone_items.begin(), lone_items.end());
+    {
+      // slice groups for sta_forward_host: each group's items in the order
+      // above (two-block items, then lone blocks)
+      const int slices = g.B * g.Hh, groups = std::min(slices, kHostGroups);
+      pl->group_slice.resize(groups + 1);
+      for (int gi = 0; gi <= groups; ++gi) pl->group_slice[gi] = (int)((long long)slices * gi / groups);
+      std::vector<int> group_of(slices);
+      for (int gi = 0; gi < groups; ++gi)
+        for (int sl = pl->group_slice[gi]; sl < pl->group_slice[gi + 1]; ++sl) group_of[sl] = gi;
+      const int n_pairs = (int)pl->work.size() - pl->n_work_lone;
+      pl->group_off.assign(groups + 1, 0);
+      pl->group_lone.assign(groups, 0);
+      for (int gi = 0; gi < groups; ++gi) {
+        pl->group_off[gi] = (int)pl->work_host.size();
+        for (int i = 0; i < (int)pl->work.size(); ++i)
+          if (group_of[pl->work[i].x] == gi) {
+            pl->work_host.push_back(pl->work[i]);
+            if (i >= n_pairs) ++pl->group_lone[gi];
+          }
+      }
+      pl->group_off[groups] = (int)pl->work_host.size();
+    }
 
     if (prob->flags & STA_PROBLEM_BACKWARD) {
       // dQ: one 128-row query block per item, heaviest heads first.
@@ -448,6 +532,7 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     pl->device = dev;
     std::vector<int32_t> cnt(pl->count);
     if (!upload(&pl->d_kv_list, pl->kv_list) || !upload(&pl->d_count, cnt) || !upload(&pl->d_work, pl->work) ||
+        !upload(&pl->d_work_host, pl->work_host) ||
         !upload(&pl->d_inv_off, pl->inv_off) || !upload(&pl->d_inv_idx, pl->inv_idx) ||
         !upload(&pl->d_work_kv, pl->work_kv) || !upload(&pl->d_work_q, pl->work_q)) {
       cudaError_t e = cudaGetLastError();
@@ -560,8 +645,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
   int *status = reinterpret_cast<int *>(ws);
 
   const void *qbase = q, *kbase = k, *vbase = v;
-  bool raster5d = pl->kv_mode == sta::kKvRaster;
-  if (!pl->tiled && !raster5d) {
+  if (!pl->tiled && pl->kv_mode != sta::kKvRaster) {
     // Tiles are not readable as TMA boxes of the raster tensor: gather Q, K
     // and V tile-major into the workspace first.
     char *dst = ws + kStatusBytes;
@@ -576,42 +660,106 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
       *base[i] = pp.dst;
     }
   }
-  CUtensorMap mq, mk, mv;
-  const bool ok = raster5d ? (make_map_raster(&mq, qbase, pl) && make_map_raster(&mk, kbase, pl) &&
-                              make_map_raster(&mv, vbase, pl))
-                           : (make_map_tiled(&mq, qbase, pl) && make_map_tiled(&mk, kbase, pl) &&
-                              make_map_tiled(&mv, vbase, pl));
-  if (!ok) return STA_ERR_CUDA;
-
-  sta::FwdParams fp{};
-  fp.g = pl->g;
-  fp.q = q, fp.o = o, fp.lse = lse;
-  fp.tiled = pl->tiled ? 1 : 0;
-  fp.nqb = pl->nqb;
-  fp.kv_list = pl->d_kv_list, fp.kv_count = pl->d_count, fp.kv_stride = pl->kv_stride;
-  fp.work = pl->d_work, fp.n_work = (int)pl->work.size(), fp.n_work_lone = pl->n_work_lone;
-  fp.scale_log2 = pl->scale * 1.4426950408889634f;
-  fp.status = status;
-  fp.wait_limit_ns = g_wait_limit_ns;
-  fp.kv_mode = raster5d ? sta::kKvRaster : sta::kKvTiled;
-  fp.piece_rows = pl->piece_rows;
-  fp.box_w = pl->box_w, fp.box_h = pl->box_h, fp.box_t = pl->box_t;
-  fp.box_panels = box_panels(pl);
-  fp.oob_coord = raster5d ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
-
   if (flags & STA_CALL_CHECK)
     if (cudaMemsetAsync(status, 0, sizeof(int), stream) != cudaSuccess) return STA_ERR_CUDA;
-  if (pl->pair) {
-    CUtensorMap mkh, mvh;
-    const bool okp = raster5d ? (make_map_raster_box(&mkh, kbase, pl, pl->kh_box[0], pl->kh_box[1], pl->kh_box[2], 2) &&
-                                 make_map_raster_box(&mvh, vbase, pl, pl->vh_box[0], pl->vh_box[1], pl->vh_box[2], 1))
-                              : (make_map_tiled_box(&mkh, kbase, pl, 64, 2) && make_map_tiled_box(&mvh, vbase, pl, 128, 1));
-    if (!okp) return STA_ERR_CUDA;
-    if (sta::launch_forward_pair(fp, mkh, mvh, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
-  } else {
-    if (sta::launch_forward(fp, mq, mk, mv, pl->num_sms, stream) != cudaSuccess) return STA_ERR_CUDA;
-  }
+  const ForwardMaps maps = forward_maps(pl, qbase, kbase, vbase);
+  if (!maps.ok) return STA_ERR_CUDA;
+  const sta_status st = enqueue_forward(pl, maps, q, o, lse, status, stream, pl->d_work, (int)pl->work.size(),
+                                        pl->n_work_lone);
+  if (st != STA_OK) return st;
   return finish_call(pl, workspace, stream, flags);
+}
+
+sta_status sta_plan_host_workspace_size(sta_plan_t pl, size_t *bytes) {
+  if (!pl || !bytes) return STA_ERR_INVALID_ARG;
+  *bytes = host_workspace(pl);
+  return STA_OK;
+}
+
+sta_status sta_forward_host(sta_plan_t pl, const void *q, const void *k, const void *v, void *o, float *lse,
+                            void *workspace, size_t ws_bytes, void *stream_, uint32_t flags) {
+  if (!pl || !q || !k || !v || !o || pl->host_only) return STA_ERR_INVALID_ARG;
+  if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < host_workspace(pl)) return STA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return STA_ERR_ALIGNMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  const size_t tb = tensor_bytes(pl), tb_r = round256(tb);
+  char *ws = static_cast<char *>(workspace);
+  char *dq = ws, *dk = ws + tb_r, *dv = ws + 2 * tb_r, *dout = ws + 3 * tb_r;
+  float *dlse = reinterpret_cast<float *>(ws + 4 * tb_r);
+  char *ws_fwd = ws + host_copies_bytes(pl);
+  const size_t fwd_bytes = fwd_workspace(pl);
+  const bool gather = !pl->tiled && pl->kv_mode != sta::kKvRaster;
+
+  if (gather || pl->pair) {
+    // no slice pipeline on these paths: whole tensors in, one sta_forward, whole outputs out
+    if ((flags & STA_CALL_CHECK) && cudaMemsetAsync(ws_fwd, 0, sizeof(int), stream) != cudaSuccess)
+      return STA_ERR_CUDA;
+    if (cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return STA_ERR_CUDA;
+    sta_status st = sta_forward(pl, dq, dk, dv, dout, lse ? dlse : nullptr, ws_fwd, fwd_bytes, stream, 0);
+    if (st != STA_OK) return st;
+    if (cudaMemcpyAsync(o, dout, tb, cudaMemcpyDeviceToHost, stream) != cudaSuccess) return STA_ERR_CUDA;
+    if (lse && cudaMemcpyAsync(lse, dlse, lse_bytes(pl), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+      return STA_ERR_CUDA;
+    return finish_call(pl, ws_fwd, stream, flags);
+  }
+
+  // Slice groups: the inputs of group g + 1 cross the bus while group g is
+  // computed, and group g's outputs come back while later groups run.
+  const int groups = (int)pl->group_slice.size() - 1;
+  const size_t slice_bytes = (size_t)pl->g.N * pl->g.d * 2, slice_lse = (size_t)pl->g.N * 4;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  std::vector<cudaEvent_t> ev(2 * groups + 2, nullptr);  // in[g], comp[g], start, done
+  auto cleanup = [&]() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+  };
+  bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess;
+  for (size_t i = 0; i < ev.size() && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+  cudaEvent_t *ev_in = ev.data(), *ev_comp = ev.data() + groups, ev_start = ev[2 * groups], ev_done = ev[2 * groups + 1];
+  int *status = reinterpret_cast<int *>(ws_fwd);
+  if (ok && (flags & STA_CALL_CHECK)) ok = cudaMemsetAsync(status, 0, sizeof(int), stream) == cudaSuccess;
+  ok = ok && cudaEventRecord(ev_start, stream) == cudaSuccess && cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+  for (int gi = 0; gi < groups && ok; ++gi) {
+    const size_t off = (size_t)pl->group_slice[gi] * slice_bytes;
+    const size_t n = (size_t)(pl->group_slice[gi + 1] - pl->group_slice[gi]) * slice_bytes;
+    ok = cudaMemcpyAsync(dq + off, static_cast<const char *>(q) + off, n, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaMemcpyAsync(dk + off, static_cast<const char *>(k) + off, n, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaMemcpyAsync(dv + off, static_cast<const char *>(v) + off, n, cudaMemcpyHostToDevice, s_in) == cudaSuccess &&
+         cudaEventRecord(ev_in[gi], s_in) == cudaSuccess;
+  }
+  const ForwardMaps maps = forward_maps(pl, dq, dk, dv);
+  ok = ok && maps.ok;
+  sta_status st = STA_OK;
+  for (int gi = 0; gi < groups && ok; ++gi) {
+    ok = cudaStreamWaitEvent(stream, ev_in[gi], 0) == cudaSuccess;
+    if (ok) {
+      st = enqueue_forward(pl, maps, dq, dout, lse ? dlse : nullptr, status, stream,
+                           pl->d_work_host + pl->group_off[gi], pl->group_off[gi + 1] - pl->group_off[gi],
+                           pl->group_lone[gi]);
+      ok = st == STA_OK && cudaEventRecord(ev_comp[gi], stream) == cudaSuccess;
+    }
+  }
+  for (int gi = 0; gi < groups && ok; ++gi) {
+    const size_t s0 = pl->group_slice[gi], ns = pl->group_slice[gi + 1] - s0;
+    ok = cudaStreamWaitEvent(s_out, ev_comp[gi], 0) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<char *>(o) + s0 * slice_bytes, dout + s0 * slice_bytes, ns * slice_bytes,
+                         cudaMemcpyDeviceToHost, s_out) == cudaSuccess;
+    if (ok && lse)
+      ok = cudaMemcpyAsync(lse + s0 * pl->g.N, dlse + s0 * pl->g.N, ns * slice_lse, cudaMemcpyDeviceToHost, s_out) ==
+           cudaSuccess;
+  }
+  ok = ok && cudaEventRecord(ev_done, s_out) == cudaSuccess && cudaStreamWaitEvent(stream, ev_done, 0) == cudaSuccess;
+  cleanup();  // destruction waits for the enqueued work on the device side
+  if (!ok) return st != STA_OK ? st : STA_ERR_CUDA;
+  return finish_call(pl, ws_fwd, stream, flags);
 }
 
 sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void *v, const void *o,

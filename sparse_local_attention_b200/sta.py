@@ -28,7 +28,8 @@ STA_CALL_CHECK = 0x1
 
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
             "sta_plan_q_tiles", "sta_plan_geometry", "sta_permute", "sta_forward", "sta_backward",
-            "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc", "sta_plan_launches"]
+            "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc", "sta_plan_launches",
+            "sta_plan_host_workspace_size", "sta_forward_host"]
 
 
 class StaError(RuntimeError):
@@ -73,6 +74,9 @@ def lib() -> ctypes.CDLL:
     L.sta_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
     L.sta_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
     L.sta_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32]
+    L.sta_plan_launches.argtypes = [vp, i32p, i32p]
+    L.sta_plan_host_workspace_size.argtypes = [vp, szp]
+    L.sta_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
     L.sta_status_string.argtypes = [ctypes.c_int]
     L.sta_status_string.restype = ctypes.c_char_p
     L.sta_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -150,6 +154,9 @@ class Plan:
         fl, bl = ctypes.c_int32(), ctypes.c_int32()
         _check(lib().sta_plan_launches(handle, ctypes.byref(fl), ctypes.byref(bl)), "sta_plan_launches")
         self.forward_launches, self.backward_launches = fl.value, bl.value  # kernels per call
+        hb = ctypes.c_size_t()
+        _check(lib().sta_plan_host_workspace_size(handle, ctypes.byref(hb)), "sta_plan_host_workspace_size")
+        self.host_workspace_bytes = hb.value
 
     def destroy(self):
         if self.handle is not None and self.handle.value:
@@ -162,8 +169,10 @@ class Plan:
         except Exception:
             pass
 
-    def workspace(self, backward=False, device=None) -> torch.Tensor:
-        n = self.bwd_workspace_bytes if backward else self.fwd_workspace_bytes
+    def workspace(self, backward=False, device=None, host=False) -> torch.Tensor:
+        """Device workspace for sta_forward, sta_backward (backward=True) or
+        sta_forward_host (host=True)."""
+        n = self.host_workspace_bytes if host else self.bwd_workspace_bytes if backward else self.fwd_workspace_bytes
         return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
@@ -235,6 +244,37 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     st = lib().sta_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
                            workspace.numel(), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_forward")
+    return o, lse
+
+
+def _expect_host(t: torch.Tensor, name: str, shape, dtype):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous host {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} cuda={t.is_cuda}")
+
+
+def sta_forward_host(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None,
+                     check: bool = False, want_lse: bool = True):
+    """Forward pass on host tensors (pin them for the copies to overlap the
+    kernels); returns host (o, lse).  The outputs are complete once `stream`
+    (default: the current stream) has passed the call."""
+    p = plan.problem
+    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _expect_host(t, nm, shape, torch.bfloat16)
+    if o is None:
+        o = torch.empty(shape, dtype=torch.bfloat16, pin_memory=q.is_pinned())
+    if lse is None and want_lse:
+        lse = torch.empty(shape[:3], dtype=torch.float32, pin_memory=q.is_pinned())
+    _expect_host(o, "o", shape, torch.bfloat16)
+    if lse is not None:
+        _expect_host(lse, "lse", shape[:3], torch.float32)
+    if workspace is None:
+        workspace = plan.workspace(host=True)
+    st = lib().sta_forward_host(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                                workspace.numel(), _stream(stream), STA_CALL_CHECK if check else 0)
+    _check(st, "sta_forward_host")
     return o, lse
 
 

@@ -198,3 +198,34 @@ def test_tiny_workload_full_oracle():
     q, k, v = make_inputs(wl)
     o, lse, _ = run_gpu(wl, q, k, v)
     compare_rows(wl, o, lse, q, k, v, np.arange(wl.B * wl.Hh * wl.N))
+
+
+# ----------------------------------------------------------------- host tensors (sta_forward_host)
+@pytest.mark.parametrize("name,pinned,cta_pair", [
+    ("d128_pair_tau384_odd_blocks", True, False),   # 2 slices, pairs and lone blocks
+    ("d64_tau192_partial_block", True, False),      # batch 2: 4 slices in 4 groups
+    ("d128_permute_fallback", True, False),         # gather path: copied whole, not pipelined
+    ("d128_pair_tau256", True, True),               # CTA-pair kernel: not pipelined
+    ("tiny_workload", False, False),                # pageable host memory
+])
+def test_forward_host_equals_device_call(name, pinned, cta_pair):
+    wl = SMALL[name]
+    q, k, v = make_inputs(wl, seed=4)
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, cta_pair=cta_pair))
+    o_dev, lse_dev = sta.sta_forward(plan, q.cuda(), k.cuda(), v.cuda(), check=True)
+    qh, kh, vh = (x.pin_memory() if pinned else x for x in (q, k, v))
+    o_h, lse_h = sta.sta_forward_host(plan, qh, kh, vh, check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(lse_h, lse_dev.cpu())
+
+
+def test_forward_host_full_scale_groups():
+    """32 slices in 8 groups of 4 (fine-tuning shapes): the pipelined host call
+    returns exactly the device call's outputs."""
+    wl = WORKLOADS["finetune"]
+    q, k, v = make_inputs(wl, seed=6)
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False))
+    o_dev, lse_dev = sta.sta_forward(plan, q.cuda(), k.cuda(), v.cuda(), check=True)
+    o_h, lse_h = sta.sta_forward_host(plan, q.pin_memory(), k.pin_memory(), v.pin_memory(), check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_h, o_dev.cpu()) and torch.equal(lse_h, lse_dev.cpu())
