@@ -84,3 +84,11 @@ def test_plan_launch_counts(tile, T, H, W, win, forward):
     assert plan.backward_launches == (4 if gather else 0) + 3
     plan_f = _create(head_dim=128, T=T, H=H, W=W, tile=tile, windows=[win])
     assert plan_f.backward_launches == 0
+
+
+def test_plan_rejects_more_rows_than_32_bit_indexing():
+    """batch * heads * T*H*W rows index the kernels' 32-bit row space; a
+    problem at 2^31 rows is refused before any table is built."""
+    with pytest.raises(sta.StaError) as e:
+        _create(batch=32, heads=1, T=64, H=1024, W=1024, tile=(1, 8, 8), windows=[(1, 1, 1)])
+    assert e.value.status == 2
