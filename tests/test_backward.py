@@ -50,6 +50,9 @@ SMALL = {
     "d64_tau384_three_blocks": Workload("b", 2, 1, 64, 12, 16, 16, (6, 8, 8), ((3, 3, 3),), backward=True),
     "d128_permute_fallback": Workload("c", 1, 2, 128, 4, 12, 8, (2, 6, 4), ((3, 1, 2), (2, 2, 2)), backward=True),
     "d64_tau192_partial_block": Workload("d", 1, 2, 64, 6, 16, 24, (3, 8, 8), ((1, 1, 3), (2, 2, 2)), backward=True),
+    # 2D (image) STA: one frame, 1 x 8 x 8 tiles
+    "d64_image_2d": Workload("e", 1, 2, 64, 1, 32, 48, (1, 8, 8), ((1, 3, 3), (1, 5, 5)), backward=True),
+    "d128_image_2d_tau256": Workload("f", 1, 1, 128, 1, 32, 64, (1, 16, 16), ((1, 1, 3),), backward=True),
 }
 
 

@@ -212,6 +212,19 @@ def test_forward_host_equals_device_call(name, pinned, cta_pair):
     wl = SMALL[name]
     q, k, v = make_inputs(wl, seed=4)
     plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, cta_pair=cta_pair))
+    _host_vs_device(plan, q, k, v, pinned)
+
+
+def test_forward_host_tile_major_tensors():
+    """sta_forward_host on a plan for tile-major tensors (the slice groups
+    are contiguous in either token order)."""
+    wl = SMALL["d64_tau384_three_blocks"]
+    q, k, v = make_inputs(wl, seed=8)
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, tiled=True))
+    _host_vs_device(plan, q, k, v, True)
+
+
+def _host_vs_device(plan, q, k, v, pinned):
     o_dev, lse_dev = sta.sta_forward(plan, q.cuda(), k.cuda(), v.cuda(), check=True)
     qh, kh, vh = (x.pin_memory() if pinned else x for x in (q, k, v))
     o_h, lse_h = sta.sta_forward_host(plan, qh, kh, vh, check=True)
