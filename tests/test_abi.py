@@ -92,3 +92,33 @@ def test_plan_rejects_more_rows_than_32_bit_indexing():
     with pytest.raises(sta.StaError) as e:
         _create(batch=32, heads=1, T=64, H=1024, W=1024, tile=(1, 8, 8), windows=[(1, 1, 1)])
     assert e.value.status == 2
+
+
+def test_c_program_on_the_abi(tmp_path):
+    """A plain C program (no Python, no torch) compiled against include/sta.h
+    and linked to libsta.so: host-only plan calls give what the binding gives."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_host"
+    lib_dir = os.path.dirname(sta.library_path())
+    subprocess.run(["gcc", "-std=c99", "-O1", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_host.c"), "-L", lib_dir, "-lsta",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    plan = _create(head_dim=128, heads=2, T=12, H=16, W=16, tile=(6, 8, 8), windows=[(3, 3, 3), (1, 1, 1)],
+                   backward=True)
+    kv = sta.sta_plan_kv_tiles(plan, 0)
+    assert got["create"] == "0"
+    assert int(got["tiles"]) == plan.n_tiles and int(got["tau"]) == plan.tile_volume
+    assert int(got["fwd_launches"]) == plan.forward_launches
+    assert int(got["bwd_launches"]) == plan.backward_launches
+    assert int(got["fwd_bytes"]) == plan.fwd_workspace_bytes and int(got["bwd_bytes"]) == plan.bwd_workspace_bytes
+    assert int(got["host_bytes"]) == plan.host_workspace_bytes
+    assert int(got["kv_entries_head0"]) == kv.numel()
+    assert int(got["kv_tile0_first"]) == int(kv[0, 0]) and int(got["kv_tile0_last"]) == int(kv[0, -1])
+    assert got["forward_on_host_plan"] == "1"
+    assert got["bad_shape"] == "2" and got["bad_head_dim"] == "3"
+    assert got["status_8"] == sta.status_string(8)
