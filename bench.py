@@ -162,6 +162,25 @@ def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
     return units_per_rank * world / (ms_max * 1e-3)
 
 
+def call_stats(per_call_ms):
+    """Median, 10th and 90th percentile of per-call times (ms)."""
+    p10, p50, p90 = np.percentile(np.asarray(per_call_ms, dtype=np.float64), [10, 50, 90])
+    return {"median": float(p50), "p10": float(p10), "p90": float(p90), "calls": len(per_call_ms)}
+
+
+def timed_calls(fn, steps: int, stream):
+    """Run fn steps times between CUDA events on stream, one event after each
+    call; return (mean ms over the whole region, per-call ms)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per_call = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[-1]) / steps, per_call
+
+
 # ---------------------------------------------------------------- CPU oracle timing
 def oracle_sample_rows(wl, n_rows: int):
     """First n_rows query rows of the first (batch, head) slice, tile by tile
@@ -191,7 +210,20 @@ def time_oracle(wl, q, k, v, target_s: float):
     oracle.forward(g, q, k, v, rows=rows)
     dt = time.perf_counter() - t0
     tflops = flops_per_row * len(rows) / dt / 1e12
-    return tflops, dt, f"{len(rows)} query rows of head 0 ({wl.keys_per_query(0)} keys each), {dt:.1f} s", oracle.threads()
+    cores = oracle.threads()
+    # the same rows on one thread, a quarter of the time budget
+    n1 = int(max(64, min(len(rows), len(rows) * target_s / 4 / max(dt * cores, 1e-3))))
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.forward(g, q, k, v, rows=rows[:n1])
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(cores)
+    extra = {"single_thread_tflops": flops_per_row * n1 / dt1 / 1e12,
+             "single_thread_sample": f"{n1} of the same rows, {dt1:.1f} s",
+             "extrapolated_full_call_s": wl.forward_flops() / (tflops * 1e12)}
+    return tflops, dt, f"{len(rows)} query rows of head 0 ({wl.keys_per_query(0)} keys each), {dt:.1f} s", cores, extra
 
 
 # ---------------------------------------------------------------- reference arm
@@ -256,19 +288,13 @@ def run_ours(args):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         clk.mark("start")
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
+        ms_rank, per_call = timed_calls(step, args.steps, stream)
         clk.mark("stop")
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    ms_rank = ev0.elapsed_time(ev1) / args.steps
     ms = max_over_ranks(dist, ms_rank)
     flops = wl.forward_flops()
     value = whole_job_rate(flops, world, ms) / 1e12
@@ -285,14 +311,11 @@ def run_ours(args):
         for _ in range(args.warmup):
             sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws)
         torch.cuda.synchronize()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        for _ in range(args.steps):
-            sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws)
-        b1.record(stream)
-        torch.cuda.synchronize()
-        bms = max_over_ranks(dist, b0.elapsed_time(b1) / args.steps)
+        bms_rank, bper_call = timed_calls(
+            lambda: sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws), args.steps, stream)
+        bms = max_over_ranks(dist, bms_rank)
         bwd = {"ms_per_step": bms, "tflops_useful": wl.backward_flops() * world / (bms * 1e-3) / 1e12,
+               "per_call_ms_rank0": call_stats(bper_call),
                "useful_flop_convention": "2.5 x forward (five GEMM-shaped products)",
                "kernels_per_step": plan.backward_launches}
         del dout, dq, dk, dv, bws
@@ -373,8 +396,8 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tflops, dt, sample, cores = time_oracle(wl, q_h, k_h, v_h, args.cpu_seconds)
-        cpu = {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+        tflops, dt, sample, cores, extra = time_oracle(wl, q_h, k_h, v_h, args.cpu_seconds)
+        cpu = {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample, **extra}
 
     clocks = clk.summary()
     if rank == 0:
@@ -384,7 +407,8 @@ def run_ours(args):
         traffic = profiled_traffic(wl.name)
         out = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms, "per_call_ms_rank0": call_stats(per_call),
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{wl.name}: {wl.description}", "useful_tflop_per_step_per_gpu": flops / 1e12,
                        "l2": "inputs 3 x %.0f MB per GPU, larger than the 126 MB L2; no flush" % (q.numel() * 2 / 1e6),

@@ -62,6 +62,8 @@ def _load():
         lib.sta_oracle_backward.restype = ctypes.c_int
         lib.sta_oracle_threads.argtypes = []
         lib.sta_oracle_threads.restype = ctypes.c_int
+        lib.sta_oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.sta_oracle_set_threads.restype = None
         _lib = lib
     return _lib
 
@@ -107,6 +109,11 @@ def _scale(geom: Geometry, scale):
 
 def threads() -> int:
     return int(_load().sta_oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads for later calls (timing only: every result is independent of it)."""
+    _load().sta_oracle_set_threads(int(n))
 
 
 def forward(geom: Geometry, q, k, v, rows=None, scale=None, exhaustive=False):

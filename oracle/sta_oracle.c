@@ -364,3 +364,13 @@ int sta_oracle_threads(void) {
   return 1;
 #endif
 }
+
+/* Set the number of OpenMP threads later calls use (n >= 1; no-op without
+ * OpenMP).  Only the timing of the oracle uses it; results do not depend on it. */
+void sta_oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

@@ -1,6 +1,7 @@
 """The N > 1 path of bench.py on the host: two gloo ranks on the CPU (no GPU,
 no data-path collective).  Checks max-over-ranks timing, the whole-job rate,
-per-rank seeds and that the reference arm runs on rank 0 only."""
+per-rank seeds and that the reference arm runs on rank 0 only; also the
+bench's host-side statistics and the oracle timing's thread switch."""
 import contextlib
 import io
 import os
@@ -63,3 +64,35 @@ def test_two_gloo_ranks():
         assert rate == 1e12 * world / 15e-3     # all ranks' units over the slowest time
         assert gathered[0] != gathered[1]       # per-rank seeds
         assert code == 0 and out == ""
+
+
+def test_call_stats_percentiles():
+    """Per-call statistics in the bench line: median and the 10th / 90th
+    percentiles (linear interpolation between order statistics)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    st = bench.call_stats([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert st["median"] == 3.0 and st["calls"] == 5
+    assert abs(st["p10"] - 1.4) < 1e-12 and abs(st["p90"] - 4.6) < 1e-12
+
+
+def test_oracle_thread_count_does_not_change_results():
+    """The bench times the oracle on all cores and on one; the result must not
+    depend on the thread count."""
+    import numpy as np
+    import oracle
+    from sparse_local_attention_b200.workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS["tiny"]
+    q, k, v = make_inputs(wl)[:3]
+    g = oracle.Geometry(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows))
+    rows = np.arange(0, wl.N, 7, dtype=np.int64)
+    cores = oracle.threads()
+    o_all, lse_all = oracle.forward(g, q, k, v, rows=rows)
+    oracle.set_threads(1)
+    try:
+        assert oracle.threads() == 1
+        o_one, lse_one = oracle.forward(g, q, k, v, rows=rows)
+    finally:
+        oracle.set_threads(cores)
+    assert oracle.threads() == cores
+    assert np.array_equal(o_all, o_one) and np.array_equal(lse_all, lse_one)
