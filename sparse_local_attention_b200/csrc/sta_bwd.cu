@@ -24,9 +24,10 @@
 //      forward KV-tile lists).  S = Q K^T and dP = dO V^T per 128-key chunk,
 //      dS in TMEM columns of its own, dQ += dS K; the next chunk's S / dP are
 //      computed while the elementwise warps work on this one.
-// Warp roles as in the forward: warps 0-7 elementwise math in two warpgroups
-// that split each chunk's columns (thread = TMEM lane = row), warp 8 TMA
-// producer, warp 9 MMA issuer.  Every wait is bounded.
+// Warp roles: NG warpgroups of elementwise warps that split each chunk's
+// columns (thread = TMEM lane = row) -- four with head dim 64, two with head
+// dim 128, whose in-place P^T / dS^T path needs 64 columns per thread -- then
+// one TMA producer warp and one MMA issuer warp.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -37,10 +38,22 @@ namespace sta {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kThreads = 320;  // 8 elementwise warps, producer, MMA issuer
-constexpr int kMathWarps = 8;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kMaxCoords = 1024;
+
+// Warp roles of the dK/dV and dQ kernels: NG warpgroups of elementwise warps
+// (warpgroup e takes columns [e kBM / NG, (e + 1) kBM / NG) of every chunk;
+// thread = TMEM lane = row), then the TMA producer warp and the MMA warp.
+// More warpgroups give each sub-partition more warps to hide the latency of
+// the elementwise pass and each thread fewer live registers.
+template <int NG>
+struct Roles {
+  static constexpr int kGroups = NG;
+  static constexpr int kMathWarps = 4 * NG;
+  static constexpr int kProducerWarp = kMathWarps, kMmaWarp = kMathWarps + 1;
+  static constexpr int kThreads = 32 * (kMathWarps + 2);
+  static constexpr int kCols = kBM / NG;  // chunk columns per warpgroup
+  static_assert(kCols % 32 == 0, "whole 32-column TMEM loads");
+};
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -126,17 +139,19 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
 }
 
 // ----------------------------------------------------------------------- 2. dK, dV
-// Warps 0-7 elementwise (warpgroup e = query columns [64 e, 64 e + 64) of each
-// 128-query chunk; thread = key row = TMEM lane), warp 8 TMA producer, warp 9
-// MMA issuer.  With head dim 64, P^T and dS^T get TMEM columns of their own,
-// so S^T / dP^T of chunk i + 1 are computed while the elementwise warps work
-// on chunk i; with head dim 128 the accumulators leave no room and P^T / dS^T
-// are written over the S^T / dP^T columns they come from.
+// Elementwise warpgroups (warpgroup e = query columns [kCW e, kCW e + kCW) of
+// each 128-query chunk, kCW = 32 with head dim 64 and 64 with head dim 128;
+// thread = key row = TMEM lane), then the TMA producer and the MMA issuer.
+// With head dim 64, P^T and dS^T get TMEM columns of their own, so S^T / dP^T
+// of chunk i + 1 are computed while the elementwise warps work on chunk i;
+// with head dim 128 the accumulators leave no room and P^T / dS^T are written
+// over the S^T / dP^T columns they come from.
 template <int D>
 struct DkvCfg {
   static constexpr uint32_t kTile = kBM * D * 2;           // one 128-row operand tile
   static constexpr uint32_t kPanel = kBM * 128;
   static constexpr bool kSep = D == 64;                    // P^T, dS^T in columns of their own
+  using R = Roles<kSep ? 4 : 2>;                           // the in-place path assumes two warpgroups
   static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr uint32_t kStage = 2 * kTile + 1024;     // Q, dO, LSE2[128], D[128]
   // barriers: st_full[S] st_empty[S] kv_full kv_free s_full s_read p_ready pd_free acc_done acc_free drain
@@ -149,11 +164,14 @@ struct DkvCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
                     const BwdParams p) {
   using C = DkvCfg<D>;
+  using R = typename C::R;
+  constexpr int kMathWarps = R::kMathWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
+  constexpr int kCW = R::kCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *k_s = smem, *v_s = smem + C::kTile;
@@ -336,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // elementwise warps: thread = key row of the block = TMEM lane; warpgroup
-    // e owns query columns [64 e, 64 e + 64)
+    // e owns query columns [kCW e, kCW e + kCW)
     const int e = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
@@ -353,11 +371,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
-        // P^T and dS^T for this warpgroup's 64 query columns, packed to bf16
+        // P^T and dS^T for this warpgroup's kCW query columns, packed to bf16
         // (query rows past the tile's end have LSE = +inf: P = dS = 0 there).
-        const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + 16 * e;
+        const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + (kCW / 4) * e;
         const float4 *dd4 = lse4 + 32;
-        uint32_t pp[2][16], pd[2][16];
+        uint32_t pp[kCW / 32][16], pd[kCW / 32][16];
         // columns q0 .. q0 + 4 n - 1 of P^T / dS^T from raw S^T / dP^T bits
         auto pds = [&](int q0, int n, const uint32_t *rs, const uint32_t *rd) {
 #pragma unroll
@@ -378,27 +396,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         };
         if constexpr (C::kSep) {
-          // S^T and dP^T are read in one batch and their columns released at
-          // once: the MMA warp computes the next chunk's while this one is done
-          uint32_t rs[2][32], rd[2][32];
+          // S^T and dP^T are read, then their columns released at once: the MMA
+          // warp computes the next chunk's while this one is done
+          // (16 columns of each at a time, so few registers stay live).
           if (okw) {
             tc_fence_after();
-            const uint32_t base = tmem + lane_off + 64 * e;
-            tmem_ld32(base + C::kTmS, rs[0]);
-            tmem_ld32(base + C::kTmS + 32, rs[1]);
-            tmem_ld32(base + C::kTmDP, rd[0]);
-            tmem_ld32(base + C::kTmDP + 32, rd[1]);
-            tmem_ld_wait();
-            if (i + 1 < nq) {
-              tc_fence_before();
-              warp_arrive(s_read, lane);
+            const uint32_t base = tmem + lane_off + kCW * e;
+#pragma unroll
+            for (int h = 0; h < kCW / 16; ++h) {
+              uint32_t rs[16], rd[16];
+              tmem_ld16(base + C::kTmS + 16 * h, rs);
+              tmem_ld16(base + C::kTmDP + 16 * h, rd);
+              tmem_ld_wait_regs(rs, rd);
+              if (h + 1 == kCW / 16 && i + 1 < nq) {
+                tc_fence_before();
+                warp_arrive(s_read, lane);
+              }
+              pds(16 * h, 4, rs, rd);
             }
-            pds(0, 8, rs[0], rd[0]);
-            pds(32, 8, rs[1], rd[1]);
           }
         } else {
           // P^T / dS^T are written over S^T / dP^T, so their columns are not
           // released early: four quarters, the next quarter's load in flight
+          static_assert(kCW == 64, "the in-place path runs two warpgroups");
           if (okw) {
             tc_fence_after();
             const uint32_t base = tmem + lane_off + 64 * e;
@@ -409,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           // both warpgroups have read their S^T / dP^T columns before either
           // writes P^T / dS^T over the first half of them
-          okw = named_bar_and(1, 256, okw);
+          okw = named_bar_and(1, 32 * kMathWarps, okw);
         }
         if (!okw) { ok = false; break; }
         if (C::kSep && gchunk > 0) {
@@ -420,29 +440,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!okf) { ok = false; break; }
           tc_fence_after();
         }
-        const uint32_t pbase = tmem + lane_off + 32 * e;
-        tmem_st16(pbase + C::kTmP, pp[0]);
-        tmem_st16(pbase + C::kTmP + 16, pp[1]);
-        tmem_st16(pbase + C::kTmDS, pd[0]);
-        tmem_st16(pbase + C::kTmDS + 16, pd[1]);
+        const uint32_t pbase = tmem + lane_off + (kCW / 2) * e;
+#pragma unroll
+        for (int h = 0; h < kCW / 32; ++h) {
+          tmem_st16(pbase + C::kTmP + 16 * h, pp[h]);
+          tmem_st16(pbase + C::kTmDS + 16 * h, pd[h]);
+        }
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(p_ready, lane);
         ++ld;
       }
       if (!ok) break;
-      // epilogue: warpgroup 0 writes dV, warpgroup 1 scale * dK (rows of this key block)
+      // epilogue: the first half of the warpgroups writes dV, the second half
+      // scale * dK (rows of this key block), each warpgroup kOut columns
       bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
       oke = __all_sync(0xffffffffu, oke);
-      if (!C::kSep) oke = named_bar_and(1, 256, oke);
+      if (!C::kSep) oke = named_bar_and(1, 32 * kMathWarps, oke);
       if (!oke) { ok = false; break; }
       tc_fence_after();
+      constexpr int kHalf = R::kGroups / 2, kOut = D / kHalf;
+      static_assert(kOut % 32 == 0, "whole 32-column TMEM loads");
+      const int which = e / kHalf, part = e % kHalf;
       const long long tok = row_valid ? token_row(g, p.tiled, bh, ktile, krow) : 0;
-      const uint32_t col = e ? C::kTmDK : C::kTmDV;
-      const float mul = e ? p.scale : 1.f;
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(e ? p.dk : p.dv) + tok * D);
+      const uint32_t col = (which ? C::kTmDK : C::kTmDV) + part * kOut;
+      const float mul = which ? p.scale : 1.f;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(which ? p.dk : p.dv) + tok * D + part * kOut);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < kOut / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + col + c * 32, r);
         tmem_ld_wait();
@@ -474,15 +499,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------- 3. dQ
-// Warps 0-7 elementwise (warpgroup e = key columns [64 e, 64 e + 64) of each
-// 128-key chunk; thread = query row), warp 8 producer, warp 9 MMA.  dS has
-// TMEM columns of its own, so S / dP of chunk j + 1 are computed while the
+// Elementwise warpgroups (warpgroup e = key columns [kCW e, kCW e + kCW) of
+// each 128-key chunk, kCW = 32 with head dim 64 and 64 with head dim 128;
+// thread = query row), then the producer and the MMA warp.  dS has TMEM
+// columns of its own, so S / dP of chunk j + 1 are computed while the
 // elementwise warps work on chunk j.
 template <int D>
 struct DqCfg {
   static constexpr uint32_t kTile = kBM * D * 2;
   static constexpr uint32_t kPanel = kBM * 128;
   static constexpr int kSlots = D == 128 ? 4 : 8;
+  using R = Roles<D == 64 ? 4 : 2>;
   // barriers: full[S] empty[S] q_full q_free s_full s_read ds_ready ds_free acc_done acc_free drain
   static constexpr int kNumBars = 2 * kSlots + 9;
   static constexpr uint32_t kSmem = (2 + kSlots) * kTile + kNumBars * 8 + 64 + 16 + kMaxCoords * 16 + 1024;
@@ -491,11 +518,14 @@ struct DqCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
                   const BwdParams p) {
   using C = DqCfg<D>;
+  using R = typename C::R;
+  constexpr int kMathWarps = R::kMathWarps, kProducerWarp = R::kProducerWarp, kMmaWarp = R::kMmaWarp;
+  constexpr int kCW = R::kCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *q_s = smem, *do_s = smem + C::kTile, *slots = smem + 2 * C::kTile;
@@ -682,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // elementwise warps: thread = query row = TMEM lane; warpgroup e owns key
-    // columns [64 e, 64 e + 64)
+    // columns [kCW e, kCW e + kCW)
     const int e = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
@@ -701,25 +731,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
-        // dS for this warpgroup's 64 key columns, packed to bf16.  S and dP are
-        // read in one batch so the MMA warp can reuse their columns at once;
+        // dS for this warpgroup's kCW key columns, packed to bf16.  S and dP
+        // are read in one batch so the MMA warp can reuse their columns at once;
         // keys past the list's end (only in the last chunk) are masked.
-        const int kvalid = it.nkeys - j * kBM - 64 * e;
-        const bool whole = kvalid >= 64;
-        uint32_t rs[2][32], rd[2][32];
-        const uint32_t base = tmem + lane_off + 64 * e;
-        tmem_ld32(base + C::kTmS, rs[0]);
-        tmem_ld32(base + C::kTmS + 32, rs[1]);
-        tmem_ld32(base + C::kTmDP, rd[0]);
-        tmem_ld32(base + C::kTmDP + 32, rd[1]);
+        const int kvalid = it.nkeys - j * kBM - kCW * e;
+        const bool whole = kvalid >= kCW;
+        uint32_t rs[kCW / 32][32], rd[kCW / 32][32];
+        const uint32_t base = tmem + lane_off + kCW * e;
+#pragma unroll
+        for (int h = 0; h < kCW / 32; ++h) tmem_ld32(base + C::kTmS + 32 * h, rs[h]);
+#pragma unroll
+        for (int h = 0; h < kCW / 32; ++h) tmem_ld32(base + C::kTmDP + 32 * h, rd[h]);
         tmem_ld_wait();
         if (j + 1 < it.nc) {
           tc_fence_before();
           warp_arrive(s_read, lane);
         }
-        uint32_t pd[2][16];
+        uint32_t pd[kCW / 32][16];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        for (int hf = 0; hf < kCW / 32; ++hf) {
           float dr[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -742,8 +772,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!okf) { ok = false; break; }
           tc_fence_after();
         }
-        tmem_st16(tmem + lane_off + C::kTmDS + 32 * e, pd[0]);
-        tmem_st16(tmem + lane_off + C::kTmDS + 32 * e + 16, pd[1]);
+#pragma unroll
+        for (int h = 0; h < kCW / 32; ++h) tmem_st16(tmem + lane_off + C::kTmDS + (kCW / 2) * e + 16 * h, pd[h]);
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(ds_ready, lane);
@@ -753,24 +783,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       oke = __all_sync(0xffffffffu, oke);
       if (!oke) { ok = false; break; }
       tc_fence_after();
-      // warpgroup e writes dQ columns [e D / 2, (e + 1) D / 2)
+      // warpgroup e writes dQ columns [e kOut, (e + 1) kOut)
+      constexpr int kOut = D / R::kGroups;
+      static_assert(kOut % 16 == 0, "whole 16-column TMEM loads");
+      constexpr int kLd = kOut < 32 ? kOut : 32;  // columns per TMEM load
       const long long tok = row_valid ? token_row(g, p.tiled, it.bh, it.tile, qrow) : 0;
-      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dq) + tok * D + e * (D / 2));
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dq) + tok * D + e * kOut);
       const float mul = p.scale;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < kOut / kLd; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_off + C::kTmDQ + e * (D / 2) + c * 32, r);
+        if constexpr (kLd == 32) {
+          tmem_ld32(tmem + lane_off + C::kTmDQ + e * kOut + c * 32, r);
+        } else {
+          tmem_ld16(tmem + lane_off + C::kTmDQ + e * kOut + c * 16, *reinterpret_cast<uint32_t(*)[16]>(r));
+        }
         tmem_ld_wait();
         if (row_valid) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < kLd / 8; ++v) {
             uint4 w;
             w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * mul, __uint_as_float(r[8 * v + 1]) * mul);
             w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * mul, __uint_as_float(r[8 * v + 3]) * mul);
             w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * mul, __uint_as_float(r[8 * v + 5]) * mul);
             w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * mul, __uint_as_float(r[8 * v + 7]) * mul);
-            dst[c * 4 + v] = w;
+            dst[c * (kLd / 8) + v] = w;
           }
         }
       }
@@ -806,9 +843,9 @@ cudaError_t launch_bwd_d(const BwdParams &p, const CUtensorMap &tq, const CUtens
   if (pre_blocks > (long long)num_sms * 16) pre_blocks = (long long)num_sms * 16;
   bwd_pre_kernel<D><<<(int)pre_blocks, 256, 0, stream>>>(p);
   const int g1 = p.n_work_kv < num_sms ? p.n_work_kv : num_sms;
-  if (g1 > 0) bwd_dkdv_kernel<D><<<g1, kThreads, DkvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  if (g1 > 0) bwd_dkdv_kernel<D><<<g1, DkvCfg<D>::R::kThreads, DkvCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   const int g2 = p.n_work_q < num_sms ? p.n_work_q : num_sms;
-  if (g2 > 0) bwd_dq_kernel<D><<<g2, kThreads, DqCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
+  if (g2 > 0) bwd_dq_kernel<D><<<g2, DqCfg<D>::R::kThreads, DqCfg<D>::kSmem, stream>>>(tq, tk, tv, tdo, p);
   return cudaGetLastError();
 }
 
