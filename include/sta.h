@@ -97,7 +97,10 @@ typedef struct sta_plan_s *sta_plan_t;
  * and, with STA_PROBLEM_BACKWARD, the inverse lists (for every key tile, the
  * query tiles whose window holds it).  Uploads them to the current device
  * (synchronous cudaMalloc + cudaMemcpy).  *out receives the plan on success and
- * is left untouched on failure. */
+ * is left untouched on failure.  Size limits (STA_ERR_SHAPE beyond them, before
+ * any table is built): batch * heads * T*H*W rows below 2^31 - 1024, and
+ * heads * tiles * (largest per-head window in tiles) list entries below
+ * 2^31 - 1, since rows and list positions are 32-bit on the device. */
 sta_status sta_plan_create(const sta_problem *problem, sta_plan_t *out);
 
 /* Free the plan and its device tables (NULL is accepted).  The caller must

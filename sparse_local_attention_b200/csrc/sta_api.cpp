@@ -349,6 +349,11 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       pl->count[h] = c;
     }
     pl->kv_stride = *std::max_element(pl->count.begin(), pl->count.end());
+    // list positions (and the inverse lists' offsets) are 32-bit on the device
+    if ((long long)g.Hh * g.n_tiles * pl->kv_stride >= (1ll << 31) - 1) {
+      delete pl;
+      return STA_ERR_SHAPE;
+    }
 
     // --- forward KV-tile lists: whole key tiles of each query tile's window,
     //     ascending tile-major index (t outer, w inner)
@@ -769,10 +774,10 @@ sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void 
     return STA_ERR_INVALID_ARG;
   if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;  // plan built without STA_PROBLEM_BACKWARD
   if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < bwd_workspace(pl)) return STA_ERR_WORKSPACE;
   const void *ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
   for (const void *ptr : ptrs)
     if (!aligned16(ptr)) return STA_ERR_ALIGNMENT;
-  if (ws_bytes < bwd_workspace(pl)) return STA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(ws);

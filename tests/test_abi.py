@@ -94,6 +94,20 @@ def test_plan_rejects_more_rows_than_32_bit_indexing():
     assert e.value.status == 2
 
 
+def test_plan_rejects_lists_past_32_bit_positions():
+    """heads * tiles * window tiles list entries are 32-bit positions on the
+    device: a plan whose lists reach 2^31 entries is refused before they are
+    built, even though its row count fits."""
+    # 1 x 1 x 376832 tokens in tiles of 8: 47104 tiles, a window over all of
+    # them gives 47104^2 = 2.2e9 list entries
+    with pytest.raises(sta.StaError) as e:
+        _create(batch=1, heads=1, T=1, H=1, W=376832, tile=(1, 1, 8), windows=[(1, 1, 47104)])
+    assert e.value.status == 2
+    # the same latent with a window of 64 tiles (3M entries) is planned
+    plan = _create(batch=1, heads=1, T=1, H=1, W=376832, tile=(1, 1, 8), windows=[(1, 1, 64)])
+    assert plan.n_tiles == 47104
+
+
 def test_c_program_on_the_abi(tmp_path):
     """A plain C program (no Python, no torch) compiled against include/sta.h
     and linked to libsta.so: host-only plan calls give what the binding gives."""
