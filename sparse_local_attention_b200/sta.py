@@ -157,6 +157,8 @@ class Plan:
         hb = ctypes.c_size_t()
         _check(lib().sta_plan_host_workspace_size(handle, ctypes.byref(hb)), "sta_plan_host_workspace_size")
         self.host_workspace_bytes = hb.value
+        # the device the tables were uploaded to; every tensor of a call must live there
+        self.device = None if problem.host_only else torch.cuda.current_device()
 
     def destroy(self):
         if self.handle is not None and self.handle.value:
@@ -171,9 +173,11 @@ class Plan:
 
     def workspace(self, backward=False, device=None, host=False) -> torch.Tensor:
         """Device workspace for sta_forward, sta_backward (backward=True) or
-        sta_forward_host (host=True)."""
+        sta_forward_host (host=True), on the plan's device."""
         n = self.host_workspace_bytes if host else self.bwd_workspace_bytes if backward else self.fwd_workspace_bytes
-        return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+        if device is None:
+            device = torch.device("cuda", self.device) if self.device is not None else "cuda"
+        return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def sta_plan_create(problem: Problem) -> Plan:
@@ -214,35 +218,65 @@ def sta_plan_q_tiles(plan: Plan, head: int):
     return off, idx[: n.value]
 
 
+def _shape(plan: Plan):
+    p = plan.problem
+    return (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+
+
+def _expect(t: torch.Tensor, name: str, shape, dtype, device: Optional[int] = None):
+    """A tensor handed to the kernels: contiguous, on the plan's CUDA device,
+    of exactly the shape and dtype the C ABI assumes (the library sees only a
+    pointer, so a wrong buffer would be read or written out of bounds)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    on_device = t.is_cuda and (device is None or t.device.index == device)
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not on_device:
+        where = f"cuda:{device}" if device is not None else "CUDA"
+        raise ValueError(f"{name}: expected contiguous {where} {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} on {t.device}")
+
+
+def _workspace(plan: Plan, ws: Optional[torch.Tensor], **kind):
+    """The caller's workspace (contiguous device memory on the plan's device;
+    its size in bytes goes to the library, which checks it), or a new one."""
+    if ws is None:
+        return plan.workspace(**kind)
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous() or (
+            plan.device is not None and ws.device.index != plan.device):
+        raise ValueError("workspace: expected a contiguous tensor on the plan's CUDA device")
+    return ws
+
+
+def _nbytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
 def sta_permute(plan: Plan, src: torch.Tensor, dst: Optional[torch.Tensor] = None, inverse: bool = False,
                 stream=None) -> torch.Tensor:
+    _expect(src, "src", _shape(plan), torch.bfloat16, plan.device)
     if dst is None:
         dst = torch.empty_like(src)
+    _expect(dst, "dst", _shape(plan), torch.bfloat16, plan.device)
     _check(lib().sta_permute(plan.handle, _ptr(src), _ptr(dst), 1 if inverse else 0, _stream(stream)), "sta_permute")
     return dst
-
-
-def _expect(t: torch.Tensor, name: str, shape, dtype):
-    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
-        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
-                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} cuda={t.is_cuda}")
 
 
 def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: Optional[torch.Tensor] = None,
                 lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None,
                 check: bool = False, want_lse: bool = True):
-    p = plan.problem
-    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    shape, dev = _shape(plan), plan.device
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
-        _expect(t, nm, shape, torch.bfloat16)
+        _expect(t, nm, shape, torch.bfloat16, dev)
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty(shape[:3], dtype=torch.float32, device=q.device)
-    if workspace is None:
-        workspace = plan.workspace(device=q.device)
+    _expect(o, "o", shape, torch.bfloat16, dev)
+    if lse is not None:
+        _expect(lse, "lse", shape[:3], torch.float32, dev)
+    workspace = _workspace(plan, workspace)
     st = lib().sta_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
-                           workspace.numel(), _stream(stream), STA_CALL_CHECK if check else 0)
+                           _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_forward")
     return o, lse
 
@@ -259,8 +293,7 @@ def sta_forward_host(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     """Forward pass on host tensors (pin them for the copies to overlap the
     kernels); returns host (o, lse).  The outputs are complete once `stream`
     (default: the current stream) has passed the call."""
-    p = plan.problem
-    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    shape = _shape(plan)
     for t, nm in ((q, "q"), (k, "k"), (v, "v")):
         _expect_host(t, nm, shape, torch.bfloat16)
     if o is None:
@@ -270,28 +303,27 @@ def sta_forward_host(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     _expect_host(o, "o", shape, torch.bfloat16)
     if lse is not None:
         _expect_host(lse, "lse", shape[:3], torch.float32)
-    if workspace is None:
-        workspace = plan.workspace(host=True)
+    workspace = _workspace(plan, workspace, host=True)
     st = lib().sta_forward_host(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
-                                workspace.numel(), _stream(stream), STA_CALL_CHECK if check else 0)
+                                _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_forward_host")
     return o, lse
 
 
 def sta_backward(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, workspace=None, stream=None,
                  check: bool = False):
-    p = plan.problem
-    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    shape, dev = _shape(plan), plan.device
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _expect(t, nm, shape, torch.bfloat16)
-    _expect(lse, "lse", shape[:3], torch.float32)
+        _expect(t, nm, shape, torch.bfloat16, dev)
+    _expect(lse, "lse", shape[:3], torch.float32, dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    if workspace is None:
-        workspace = plan.workspace(backward=True, device=q.device)
+    for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _expect(t, nm, shape, torch.bfloat16, dev)
+    workspace = _workspace(plan, workspace, backward=True)
     st = lib().sta_backward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                            _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream),
+                            _ptr(dk), _ptr(dv), _ptr(workspace), _nbytes(workspace), _stream(stream),
                             STA_CALL_CHECK if check else 0)
     _check(st, "sta_backward")
     return dq, dk, dv
@@ -302,14 +334,15 @@ def sta_backward_noalloc(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv
     """sta_backward with the library's fixed device scratch instead of a
     workspace (see include/sta.h).  Output tensors may be passed in; if they
     are not, they are created here by the caller's allocator (torch)."""
-    p = plan.problem
-    shape = (p.batch, p.heads, p.T * p.H * p.W, p.head_dim)
+    shape, dev = _shape(plan), plan.device
     for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _expect(t, nm, shape, torch.bfloat16)
-    _expect(lse, "lse", shape[:3], torch.float32)
+        _expect(t, nm, shape, torch.bfloat16, dev)
+    _expect(lse, "lse", shape[:3], torch.float32, dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _expect(t, nm, shape, torch.bfloat16, dev)
     st = lib().sta_backward_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                     _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_backward_noalloc")

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from sparse_local_attention_b200 import sta
 
@@ -106,6 +107,32 @@ def test_plan_rejects_lists_past_32_bit_positions():
     # the same latent with a window of 64 tiles (3M entries) is planned
     plan = _create(batch=1, heads=1, T=1, H=1, W=376832, tile=(1, 1, 8), windows=[(1, 1, 64)])
     assert plan.n_tiles == 47104
+
+
+def test_binding_refuses_buffers_the_kernels_cannot_use():
+    """The library sees only pointers, so the binding checks every tensor it
+    passes (shape, dtype, contiguity, CUDA residency) before any call: host
+    tensors, wrong shapes and non-tensors are refused without reaching it."""
+    plan = _create(backward=True)
+    shape = (1, 1, 4 * 8 * 8, 64)
+    x = torch.zeros(shape, dtype=torch.bfloat16)
+    lse = torch.zeros(shape[:3], dtype=torch.float32)
+    with pytest.raises(ValueError, match="q: expected contiguous"):
+        sta.sta_forward(plan, x, x, x)
+    with pytest.raises(ValueError, match="src: expected contiguous"):
+        sta.sta_permute(plan, x)
+    with pytest.raises(ValueError, match="q: expected contiguous"):
+        sta.sta_backward(plan, x, x, x, x, lse, x)
+    with pytest.raises(ValueError, match="expected contiguous"):
+        sta.sta_forward(plan, x[..., :32], x, x)          # wrong head dim
+    with pytest.raises(ValueError, match="expected contiguous"):
+        sta.sta_forward(plan, x.transpose(2, 3).contiguous().transpose(2, 3), x, x)  # strided
+    with pytest.raises(TypeError):
+        sta.sta_forward(plan, [0.0] * 64, x, x)
+    # host tensors of the right shape are what sta_forward_host takes; its
+    # device workspace is checked too
+    with pytest.raises(ValueError, match="workspace"):
+        sta.sta_forward_host(plan, x, x, x, workspace=torch.zeros(16, dtype=torch.uint8))
 
 
 def test_c_program_on_the_abi(tmp_path):
