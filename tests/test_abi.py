@@ -135,6 +135,92 @@ def test_binding_refuses_buffers_the_kernels_cannot_use():
         sta.sta_forward_host(plan, x, x, x, workspace=torch.zeros(16, dtype=torch.uint8))
 
 
+class _OnCuda0(torch.Tensor):
+    """A host tensor that reports itself as living on cuda:0 (to exercise the
+    binding's marshalling of device calls without a GPU)."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+    @property
+    def device(self):
+        return torch.device("cuda", 0)
+
+
+class _OnCuda1(_OnCuda0):
+    @property
+    def device(self):
+        return torch.device("cuda", 1)
+
+
+class _RecordingLib:
+    """Stands in for libsta.so: records each call's arguments, returns STA_OK."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def call(*args):
+            self.calls.append((name, args))
+            return 0
+        return call
+
+
+def test_binding_passes_valid_device_buffers_through(monkeypatch):
+    """Valid device-side calls pass the binding's checks and reach the library
+    with the tensors' own pointers and the workspace size in bytes; buffers of
+    another shape, dtype or device are refused."""
+    plan = _create(backward=True)
+    plan.device = 0  # as if the tables had been uploaded to cuda:0
+    shape = (1, 1, 4 * 8 * 8, 64)
+    dev = lambda t: t.as_subclass(_OnCuda0)
+    q, k, v, o, do = (dev(torch.zeros(shape, dtype=torch.bfloat16)) for _ in range(5))
+    lse = dev(torch.zeros(shape[:3], dtype=torch.float32))
+    ws = dev(torch.zeros(100, dtype=torch.float32))  # 400 bytes
+    rec = _RecordingLib()
+    monkeypatch.setattr(sta, "lib", lambda: rec)
+
+    sta.sta_forward(plan, q, k, v, o, lse, ws, stream=0, check=True)
+    name, args = rec.calls[-1]
+    assert name == "sta_forward"
+    assert [a.value for a in args[1:7]] == [t.data_ptr() for t in (q, k, v, o, lse, ws)]
+    assert args[7] == 400 and args[9] == sta.STA_CALL_CHECK
+
+    dq, dk, dv = sta.sta_backward(plan, q, k, v, o, lse, do, workspace=ws, stream=0)
+    name, args = rec.calls[-1]
+    assert name == "sta_backward" and args[11] == 400
+    assert [a.value for a in args[7:10]] == [t.data_ptr() for t in (dq, dk, dv)]
+    assert all(t.shape == q.shape and t.dtype == torch.bfloat16 for t in (dq, dk, dv))
+
+    dst = sta.sta_permute(plan, q, stream=0, inverse=True)
+    name, args = rec.calls[-1]
+    assert name == "sta_permute" and args[2].value == dst.data_ptr() and args[3] == 1
+
+    qh = torch.zeros(shape, dtype=torch.bfloat16)
+    oh, lh = sta.sta_forward_host(plan, qh, qh, qh, workspace=ws, stream=0)
+    name, args = rec.calls[-1]
+    assert name == "sta_forward_host" and args[7] == 400
+    assert oh.shape == shape and not oh.is_cuda and lh.shape == shape[:3]
+
+    n = len(rec.calls)
+    bad = [
+        dict(o=dev(torch.zeros(shape[:3] + (32,), dtype=torch.bfloat16))),   # o: wrong head dim
+        dict(lse=dev(torch.zeros(shape[:3], dtype=torch.bfloat16))),         # lse: wrong dtype
+        dict(o=torch.zeros(shape, dtype=torch.bfloat16).as_subclass(_OnCuda1)),  # o: another GPU
+        dict(workspace=torch.zeros(400, dtype=torch.uint8)),                  # host workspace
+    ]
+    for kw in bad:
+        args = dict(o=o, lse=lse, workspace=ws)
+        args.update(kw)
+        with pytest.raises(ValueError):
+            sta.sta_forward(plan, q, k, v, stream=0, **args)
+    with pytest.raises(ValueError, match="dk"):
+        sta.sta_backward(plan, q, k, v, o, lse, do, dk=dev(torch.zeros(shape, dtype=torch.float32)),
+                         workspace=ws, stream=0)
+    assert len(rec.calls) == n  # none of them reached the library
+
+
 def test_c_program_on_the_abi(tmp_path):
     """A plain C program (no Python, no torch) compiled against include/sta.h
     and linked to libsta.so: host-only plan calls give what the binding gives."""
