@@ -156,10 +156,22 @@ def max_over_ranks(dist, x: float, device="cuda") -> float:
     return float(t.item())
 
 
-def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
-    """Throughput of the whole job: the units every rank processed over the
-    slowest rank's time (weak scaling: each rank has its own problem)."""
-    return units_per_rank * world / (ms_max * 1e-3)
+def rank_share(wl, world: int, rank: int, shard: str):
+    """This rank's problem: (workload, heads or None, the job's useful forward
+    FLOPs per step, scaling).
+
+    shard "problem": every rank runs the whole workload on inputs seeded by
+    its rank (weak scaling: per-GPU work fixed as N grows).  shard "heads":
+    the ranks split one problem's heads, longest-processing-time by keys per
+    query, and each keeps its heads of the same seeded inputs (strong
+    scaling: the job is fixed)."""
+    from sparse_local_attention_b200.sharding import head_costs, partition_heads, shard_workload
+    if shard == "heads":
+        parts = partition_heads(head_costs(wl), world)
+        if any(not p for p in parts):
+            raise SystemExit(f"--shard heads: {wl.Hh} heads cannot give each of {world} ranks at least one")
+        return shard_workload(wl, parts[rank]), parts[rank], wl.forward_flops(), "strong"
+    return wl, None, wl.forward_flops() * world, "weak"
 
 
 def call_stats(per_call_ms):
@@ -264,13 +276,22 @@ def run_reference(args):
 def run_ours(args):
     from sparse_local_attention_b200 import sta
 
+    from sparse_local_attention_b200.sharding import select_heads
+
     world, rank, local = dist_env()
+    wl_job = WORKLOADS[args.workload]
+    wl, heads, job_flops, scaling = rank_share(wl_job, world, rank, args.shard)
     dist = init_dist(world, local)
     torch.cuda.set_device(local)
-    wl = WORKLOADS[args.workload]
     pk, pk_kind = peaks()
 
-    q_h, k_h, v_h = (x.pin_memory() for x in make_inputs(wl, seed=rank))
+    def inputs(with_dout=False):
+        """This rank's inputs: its own seeded problem, or its heads of the job's."""
+        if heads is None:
+            return make_inputs(wl, with_dout=with_dout, seed=rank)
+        return tuple(select_heads(x, heads) for x in make_inputs(wl_job, with_dout=with_dout, seed=0))
+
+    q_h, k_h, v_h = (x.pin_memory() for x in inputs())
     q, k, v = (x.cuda() for x in (q_h, k_h, v_h))
     plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=wl.backward))
     o = torch.empty_like(q)
@@ -296,14 +317,14 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     ms = max_over_ranks(dist, ms_rank)
-    flops = wl.forward_flops()
-    value = whole_job_rate(flops, world, ms) / 1e12
+    flops = wl.forward_flops()  # this rank's
+    value = job_flops / (ms * 1e-3) / 1e12
     launches_per_step = plan.forward_launches  # kernels one sta_forward call enqueues
 
     # --- backward (fine-tuning workloads): dQ, dK, dV from the same inputs
     bwd = None
     if wl.backward:
-        do_h = make_inputs(wl, with_dout=True, seed=rank)[3]
+        do_h = inputs(with_dout=True)[3]
         dout = do_h.cuda()
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         bws = plan.workspace(backward=True)
@@ -314,7 +335,7 @@ def run_ours(args):
         bms_rank, bper_call = timed_calls(
             lambda: sta.sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, bws), args.steps, stream)
         bms = max_over_ranks(dist, bms_rank)
-        bwd = {"ms_per_step": bms, "tflops_useful": wl.backward_flops() * world / (bms * 1e-3) / 1e12,
+        bwd = {"ms_per_step": bms, "tflops_useful": 2.5 * job_flops / (bms * 1e-3) / 1e12,
                "per_call_ms_rank0": call_stats(bper_call),
                "useful_flop_convention": "2.5 x forward (five GEMM-shaped products)",
                "kernels_per_step": plan.backward_launches}
@@ -377,7 +398,7 @@ def run_ours(args):
 
     # --- dense full-attention baseline on the same shapes (library SDPA)
     dense = None
-    if not args.no_dense and rank == 0:
+    if not args.no_dense and rank == 0 and heads is None:
         torch.backends.cuda.enable_flash_sdp(True)
         for _ in range(2):
             torch.nn.functional.scaled_dot_product_attention(q, k, v)
@@ -408,17 +429,19 @@ def run_ours(args):
         out = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "per_call_ms_rank0": call_stats(per_call),
-            "higher_is_better": True, "scaling": "weak",
+            "higher_is_better": True, "scaling": scaling,
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: {wl.description}", "useful_tflop_per_step_per_gpu": flops / 1e12,
+            "config": {"workload": f"{wl_job.name}: {wl_job.description}",
+                       "useful_tflop_per_step": job_flops / 1e12, "useful_tflop_per_step_rank0": flops / 1e12,
                        "l2": "inputs 3 x %.0f MB per GPU, larger than the 126 MB L2; no flush" % (q.numel() * 2 / 1e6),
-                       "parallelism": f"independent problem per GPU x{world}"},
+                       "parallelism": (f"independent problem per GPU x{world}" if heads is None else
+                                       f"heads split over {world} GPUs by keys per query (rank 0: heads {heads})")},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{pk_kind} {peak_key}",
                          "kernel": "sta_fwd_kernel (one forward call: %d launch(es), timed together)" % launches_per_step,
                          "per": "forward call"},
-            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+            "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
@@ -446,6 +469,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=384)
+    ap.add_argument("--shard", default="problem", choices=["problem", "heads"],
+                    help="problem: one independent problem per GPU (weak scaling); "
+                         "heads: one problem's heads split over the GPUs (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -11,6 +11,8 @@ import sys
 import torch
 import torch.multiprocessing as mp
 
+from sparse_local_attention_b200.workloads import WORKLOADS
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -32,7 +34,13 @@ def _worker(rank: int, world: int, port: int, results):
     try:
         # each rank times its own problem; the job's time is the slowest rank's
         ms = bench.max_over_ranks(dist, 10.0 + 5.0 * rank, device="cpu")
-        rate = bench.whole_job_rate(1e12, w, ms)
+        _, _, job_flops, _ = bench.rank_share(WORKLOADS["tiny"], w, r, "problem")
+        rate = job_flops / (ms * 1e-3)
+        # one problem's heads split over the ranks: every head on exactly one rank
+        sub, heads, job_h, scaling = bench.rank_share(WORKLOADS["dit720p_perhead"], w, r, "heads")
+        mine = torch.zeros(24)
+        mine[heads] = 1.0
+        dist.all_reduce(mine)
         # ranks draw different inputs (independent problems)
         q = make_inputs(WORKLOADS["tiny"], seed=r)[0]
         first = torch.tensor([float(q.float().sum())])
@@ -46,7 +54,8 @@ def _worker(rank: int, world: int, port: int, results):
         else:
             code = 0
         dist.barrier()
-        results[rank] = (w, r, ms, rate, [float(x) for x in gathered], code, out.getvalue())
+        results[rank] = (w, r, ms, rate, [float(x) for x in gathered], code, out.getvalue(),
+                         mine.tolist(), sub.forward_flops(), job_h, scaling)
     finally:
         dist.destroy_process_group()
 
@@ -58,10 +67,15 @@ def test_two_gloo_ranks():
     mp.start_processes(_worker, args=(world, _free_port(), results), nprocs=world, start_method="spawn", join=True)
     assert sorted(results.keys()) == [0, 1]
     for rank in range(world):
-        w, r, ms, rate, gathered, code, out = results[rank]
+        w, r, ms, rate, gathered, code, out, cover, sub_flops, job_h, scaling = results[rank]
         assert (w, r) == (world, rank)
         assert ms == 15.0                       # max over ranks, same on every rank
-        assert rate == 1e12 * world / 15e-3     # all ranks' units over the slowest time
+        tiny = WORKLOADS["tiny"].forward_flops()
+        assert rate == tiny * world / 15e-3     # all ranks' units over the slowest time
+        assert cover == [1.0] * 24              # each head on exactly one rank
+        full = WORKLOADS["dit720p_perhead"].forward_flops()
+        assert job_h == full and scaling == "strong"
+        assert sub_flops == full / world        # three window classes split evenly
         assert gathered[0] != gathered[1]       # per-rank seeds
         assert code == 0 and out == ""
 
