@@ -9,6 +9,8 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
+from collections import OrderedDict
 from dataclasses import dataclass, field
 from typing import Optional, Sequence
 
@@ -161,7 +163,12 @@ class Plan:
         self.device = None if problem.host_only else torch.cuda.current_device()
 
     def destroy(self):
+        """Free the plan.  Its device tables are read by every launch that uses
+        it, so the plan's device is synchronised first: no such launch can
+        still be running when they are freed."""
         if self.handle is not None and self.handle.value:
+            if self.device is not None:
+                torch.cuda.synchronize(self.device)
             _check(lib().sta_plan_destroy(self.handle), "sta_plan_destroy")
         self.handle = None
 
@@ -270,7 +277,7 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     if o is None:
         o = torch.empty_like(q)
     if lse is None and want_lse:
-        lse = torch.empty(shape[:3], dtype=torch.float32, device=q.device)
+        lse = q.new_empty(shape[:3], dtype=torch.float32)
     _expect(o, "o", shape, torch.bfloat16, dev)
     if lse is not None:
         _expect(lse, "lse", shape[:3], torch.float32, dev)
@@ -353,12 +360,71 @@ def sta_set_wait_limit_ns(ns: int):
     lib().sta_set_wait_limit_ns(int(ns))
 
 
+class _SlidingTileAttention(torch.autograd.Function):
+    """O = STA(q, k, v) with its gradient: sta_forward saves LSE, and the
+    backward is one sta_backward call (the plan must carry the inverse lists)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, plan):
+        o, lse = sta_forward(plan, q, k, v)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.plan = plan
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = sta_backward(ctx.plan, q, k, v, o, lse, do.contiguous())
+        return dq, dk, dv, None
+
+
+_PLANS: "OrderedDict[tuple, Plan]" = OrderedDict()
+_PLANS_LOCK = threading.Lock()
+PLAN_CACHE_SIZE = 16
+
+
+def cached_plan(problem: Problem) -> Plan:
+    """The plan of `problem` on the current device, built on first use and
+    kept (the PLAN_CACHE_SIZE most recently used).  A plan that leaves the
+    cache is freed once nothing refers to it any more (an autograd graph may
+    still hold it for its backward)."""
+    key = (problem.batch, problem.heads, problem.head_dim, problem.T, problem.H, problem.W, tuple(problem.tile),
+           tuple(tuple(int(x) for x in w) for w in problem.windows), float(problem.scale), problem.backward,
+           problem.tiled, problem.cta_pair, torch.cuda.current_device())
+    with _PLANS_LOCK:
+        plan = _PLANS.get(key)
+        if plan is not None:
+            _PLANS.move_to_end(key)
+            return plan
+        plan = sta_plan_create(problem)
+        _PLANS[key] = plan
+        while len(_PLANS) > PLAN_CACHE_SIZE:
+            _PLANS.popitem(last=False)
+        return plan
+
+
+def _per_head(windows, heads: int):
+    """One (w_t, w_h, w_w) for every head, or one per head."""
+    if len(windows) == 3 and all(isinstance(x, int) for x in windows):
+        return tuple([tuple(int(x) for x in windows)] * heads)
+    if len(windows) != heads:
+        raise ValueError(f"{len(windows)} windows for {heads} heads")
+    return tuple(tuple(int(x) for x in w) for w in windows)
+
+
 def sliding_tile_attention(q, k, v, T, H, W, tile, windows, scale=0.0):
-    """One-shot convenience: plan + forward (the plan is rebuilt every call)."""
+    """Sliding Tile Attention of bf16 [batch, heads, T*H*W, d] tensors in
+    raster token order; returns O (same shape).  `windows`: one (w_t, w_h, w_w)
+    in tiles for every head, or one per head.  Differentiable: when q, k or v
+    requires a gradient, the backward runs sta_backward.  The plan comes from
+    a small cache keyed by the problem, so repeated calls do not rebuild it.
+    Non-contiguous inputs are made contiguous first."""
     B, Hh, N, d = q.shape
-    plan = sta_plan_create(Problem(B, Hh, d, T, H, W, tuple(tile), tuple(tuple(w) for w in windows), scale))
-    try:
-        return sta_forward(plan, q, k, v)
-    finally:
-        torch.cuda.current_stream().synchronize()
-        plan.destroy()
+    if N != T * H * W:
+        raise ValueError(f"token count {N} != T*H*W = {T * H * W}")
+    plan = cached_plan(Problem(B, Hh, d, T, H, W, tuple(tile), _per_head(windows, Hh), scale, backward=True))
+    q, k, v = (t.contiguous() for t in (q, k, v))
+    if torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v)):
+        return _SlidingTileAttention.apply(q, k, v, plan)
+    o, _ = sta_forward(plan, q, k, v, want_lse=False)
+    return o

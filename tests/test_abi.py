@@ -249,3 +249,57 @@ def test_c_program_on_the_abi(tmp_path):
     assert got["forward_on_host_plan"] == "1"
     assert got["bad_shape"] == "2" and got["bad_head_dim"] == "3"
     assert got["status_8"] == sta.status_string(8)
+
+
+def test_autograd_and_plan_cache_marshalling(monkeypatch):
+    """sliding_tile_attention: the forward is one sta_forward call, the
+    backward one sta_backward call on the saved q, k, v, o, lse with the
+    incoming gradient, and its dq, dk, dv are the gradients autograd returns;
+    plans come from a bounded cache keyed by the problem.  (Fake cuda:0
+    tensors and a recording library: no GPU.)"""
+    from collections import OrderedDict
+    rec = _RecordingLib()
+    monkeypatch.setattr(sta, "lib", lambda: rec)
+    monkeypatch.setattr(sta, "_PLANS", OrderedDict())
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
+    monkeypatch.setattr(sta, "_stream", lambda stream: ctypes.c_void_p(0))
+
+    def expect_shape(t, name, shape, dtype, device=None):
+        # autograd hands saved tensors back as plain (host) tensors, so only
+        # shape and dtype are checked here; the device checks have their own tests
+        assert tuple(t.shape) == tuple(shape) and t.dtype == dtype, name
+    monkeypatch.setattr(sta, "_expect", expect_shape)
+    monkeypatch.setattr(sta.Plan, "workspace",
+                        lambda self, **kw: torch.zeros(256, dtype=torch.uint8).as_subclass(_OnCuda0))
+    T, H, W, tile = 4, 8, 8, (2, 4, 4)
+    shape = (1, 2, T * H * W, 64)
+    q, k, v = (torch.randn(shape).to(torch.bfloat16).as_subclass(_OnCuda0).requires_grad_() for _ in range(3))
+
+    o = sta.sliding_tile_attention(q, k, v, T, H, W, tile, (3, 3, 3))
+    assert [c[0] for c in rec.calls].count("sta_plan_create") == 1
+    fwd = [c for c in rec.calls if c[0] == "sta_forward"][-1][1]
+    assert [a.value for a in fwd[1:4]] == [t.data_ptr() for t in (q, k, v)]
+    assert fwd[4].value == o.data_ptr() and fwd[5].value is not None  # LSE kept for the backward
+
+    do = torch.randn(shape).to(torch.bfloat16).as_subclass(_OnCuda0)
+    grads = torch.autograd.grad(o, (q, k, v), grad_outputs=do)
+    bwd = [c for c in rec.calls if c[0] == "sta_backward"][-1][1]
+    assert [a.value for a in bwd[1:5]] == [t.data_ptr() for t in (q, k, v, o)]
+    assert bwd[5].value == fwd[5].value and bwd[6].value == do.data_ptr()
+    assert [a.value for a in bwd[7:10]] == [g.data_ptr() for g in grads]
+
+    # the same problem reuses its plan; other windows get their own; no grad -> no LSE
+    with torch.no_grad():
+        sta.sliding_tile_attention(q, k, v, T, H, W, tile, [(3, 3, 3), (3, 3, 3)])
+        assert [c[0] for c in rec.calls].count("sta_plan_create") == 1
+        assert [c for c in rec.calls if c[0] == "sta_forward"][-1][1][5] is None
+        sta.sliding_tile_attention(q, k, v, T, H, W, tile, [(1, 1, 1), (3, 3, 3)])
+    assert [c[0] for c in rec.calls].count("sta_plan_create") == 2
+    monkeypatch.setattr(sta, "PLAN_CACHE_SIZE", 2)
+    with torch.no_grad():
+        for w in ((1, 1, 1), (2, 2, 2), (1, 2, 1)):
+            sta.sliding_tile_attention(q, k, v, T, H, W, tile, w)
+    assert len(sta._PLANS) == 2
+    with pytest.raises(ValueError):
+        sta.sliding_tile_attention(q, k, v, T, H, W, tile, [(3, 3, 3)] * 3)  # 3 windows, 2 heads

@@ -143,3 +143,27 @@ def test_gradient_identities_full_scale(name):
     k_eq = k[:, :, :1].expand_as(k).contiguous()
     _, _, (dq0, _, _) = run_fwd_bwd(wl, q, k_eq, v, do)
     assert dq0.float().abs().max() < 2e-3, float(dq0.float().abs().max())
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny"].with_(backward=True), SMALL["d128_tau64"]], ids=lambda w: w.name)
+def test_autograd_function_matches_the_abi_calls(wl):
+    """sliding_tile_attention under autograd: its O equals sta_forward's and the
+    gradients of sum(O * dO) equal sta_backward's for the same dO, bit for bit
+    (the same deterministic kernels on the same inputs); without gradients it
+    returns the same O."""
+    q, k, v, do = (x.cuda() for x in make_inputs(wl, with_dout=True, seed=5))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=True))
+    o_ref, lse_ref = sta.sta_forward(plan, q, k, v, check=True)
+    g_ref = sta.sta_backward(plan, q, k, v, o_ref, lse_ref, do, check=True)
+    qa, ka, va = (x.clone().requires_grad_() for x in (q, k, v))
+    o = sta.sliding_tile_attention(qa, ka, va, wl.T, wl.H, wl.W, wl.tile, wl.windows)
+    (o.float() * do.float()).sum().backward()
+    torch.cuda.synchronize()
+    assert torch.equal(o.detach(), o_ref)
+    for name, got, ref in zip(("dq", "dk", "dv"), (qa.grad, ka.grad, va.grad), g_ref):
+        assert torch.equal(got, ref), name
+    with torch.no_grad():
+        o_plain = sta.sliding_tile_attention(q, k, v, wl.T, wl.H, wl.W, wl.tile, wl.windows)
+    torch.cuda.synchronize()
+    assert torch.equal(o_plain, o_ref)
+    plan.destroy()
