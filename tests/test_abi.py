@@ -221,6 +221,24 @@ def test_binding_passes_valid_device_buffers_through(monkeypatch):
     assert len(rec.calls) == n  # none of them reached the library
 
 
+def test_planner_reports_out_of_memory(tmp_path):
+    """A host allocation failure inside sta_plan_create (injected by capping
+    the process's address space, in a C program of its own) is STA_ERR_OOM,
+    leaves the output handle untouched, and the library keeps working."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_oom"
+    lib_dir = os.path.dirname(sta.library_path())
+    subprocess.run(["gcc", "-std=gnu99", "-O1", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_oom.c"), "-L", lib_dir, "-lsta",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    assert got == {"big_status": "6", "big_untouched": "1", "small_status": "0"}
+
+
 def test_c_program_on_the_abi(tmp_path):
     """A plain C program (no Python, no torch) compiled against include/sta.h
     and linked to libsta.so: host-only plan calls give what the binding gives."""
