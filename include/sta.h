@@ -129,6 +129,28 @@ sta_status sta_plan_q_tiles(sta_plan_t plan, int32_t head, int32_t *offsets, int
 /* Number of tiles of the plan's grid and tokens per tile. */
 sta_status sta_plan_geometry(sta_plan_t plan, int32_t *n_tiles, int32_t *tile_volume);
 
+/* Host copy of one of the plan's work lists, for tests and tooling.  Rows of a
+ * tile are cut into blocks of 128 (the last one partial): block b of tile t of
+ * a (batch, head) slice s = batch * heads + head is numbered t * nb + b, with
+ * nb = ceil(tile_volume / 128).
+ *   which = STA_WORK_FORWARD (0): the forward's items, 4 int32 each:
+ *       (slice, block A, block B or -1, 0).  A and B attend to the same key
+ *       tiles; items with B = -1 (lone blocks) come last, *n_lone of them.
+ *   which = STA_WORK_FORWARD_HOST (1): the same items in sta_forward_host's
+ *       order (slice groups one after another), 4 int32 each.
+ *   which = STA_WORK_DKDV (2) / STA_WORK_DQ (3): the backward's items, 2 int32
+ *       each: (slice, key block) / (slice, query block); empty for a plan
+ *       built without STA_PROBLEM_BACKWARD.
+ * *n_items receives the item count (out may be NULL to query it; otherwise
+ * cap_items must be >= *n_items, else STA_ERR_INVALID_ARG).  n_lone may be
+ * NULL.  This call has no counterpart in the paper. */
+#define STA_WORK_FORWARD 0
+#define STA_WORK_FORWARD_HOST 1
+#define STA_WORK_DKDV 2
+#define STA_WORK_DQ 3
+sta_status sta_plan_work_items(sta_plan_t plan, int32_t which, int32_t *out, size_t cap_items, size_t *n_items,
+                               int32_t *n_lone);
+
 /* Number of kernels one sta_forward / sta_backward call of this plan enqueues
  * on its stream (the status-word memset of STA_CALL_CHECK is not counted;
  * `backward` is 0 for a plan built without STA_PROBLEM_BACKWARD).  For sizing

@@ -571,6 +571,31 @@ sta_status sta_plan_geometry(sta_plan_t pl, int32_t *n_tiles, int32_t *tile_volu
   return STA_OK;
 }
 
+sta_status sta_plan_work_items(sta_plan_t pl, int32_t which, int32_t *out, size_t cap_items, size_t *n_items,
+                               int32_t *n_lone) {
+  if (!pl || !n_items) return STA_ERR_INVALID_ARG;
+  if (n_lone) *n_lone = pl->n_work_lone;
+  if (which == STA_WORK_FORWARD || which == STA_WORK_FORWARD_HOST) {
+    const std::vector<int4> &w = which == STA_WORK_FORWARD ? pl->work : pl->work_host;
+    *n_items = w.size();
+    if (!out) return STA_OK;
+    if (cap_items < w.size()) return STA_ERR_INVALID_ARG;
+    for (size_t i = 0; i < w.size(); ++i) {
+      out[4 * i] = w[i].x, out[4 * i + 1] = w[i].y, out[4 * i + 2] = w[i].z, out[4 * i + 3] = w[i].w;
+    }
+    return STA_OK;
+  }
+  if (which == STA_WORK_DKDV || which == STA_WORK_DQ) {
+    const std::vector<int2> &w = which == STA_WORK_DKDV ? pl->work_kv : pl->work_q;
+    *n_items = w.size();
+    if (!out) return STA_OK;
+    if (cap_items < w.size()) return STA_ERR_INVALID_ARG;
+    for (size_t i = 0; i < w.size(); ++i) out[2 * i] = w[i].x, out[2 * i + 1] = w[i].y;
+    return STA_OK;
+  }
+  return STA_ERR_INVALID_ARG;
+}
+
 sta_status sta_plan_launches(sta_plan_t pl, int32_t *forward, int32_t *backward) {
   if (!pl) return STA_ERR_INVALID_ARG;
   const int n_work = (int)pl->work.size();

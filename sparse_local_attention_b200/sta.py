@@ -31,7 +31,8 @@ STA_CALL_CHECK = 0x1
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
             "sta_plan_q_tiles", "sta_plan_geometry", "sta_permute", "sta_forward", "sta_backward",
             "sta_status_string", "sta_set_wait_limit_ns", "sta_backward_noalloc", "sta_plan_launches",
-            "sta_plan_host_workspace_size", "sta_forward_host"]
+            "sta_plan_host_workspace_size", "sta_forward_host", "sta_plan_work_items"]
+STA_WORK_FORWARD, STA_WORK_FORWARD_HOST, STA_WORK_DKDV, STA_WORK_DQ = 0, 1, 2, 3
 
 
 class StaError(RuntimeError):
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.sta_plan_launches.argtypes = [vp, i32p, i32p]
     L.sta_plan_host_workspace_size.argtypes = [vp, szp]
     L.sta_forward_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.c_uint32]
+    L.sta_plan_work_items.argtypes = [vp, ctypes.c_int32, i32p, sz, szp, i32p]
     L.sta_status_string.argtypes = [ctypes.c_int]
     L.sta_status_string.restype = ctypes.c_char_p
     L.sta_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -211,6 +213,19 @@ def sta_plan_kv_tiles(plan: Plan, head: int) -> torch.Tensor:
     _check(lib().sta_plan_kv_tiles(plan.handle, head, ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
                                    n.value, ctypes.byref(n)), "sta_plan_kv_tiles")
     return out.view(plan.n_tiles, -1)
+
+
+def sta_plan_work_items(plan: Plan, which: int):
+    """(items, n_lone): one of the plan's work lists as an int32 [n, 4]
+    (forward lists) or [n, 2] (backward lists) host tensor; see include/sta.h."""
+    n, lone = ctypes.c_size_t(), ctypes.c_int32()
+    _check(lib().sta_plan_work_items(plan.handle, which, None, 0, ctypes.byref(n), ctypes.byref(lone)),
+           "sta_plan_work_items")
+    width = 4 if which in (STA_WORK_FORWARD, STA_WORK_FORWARD_HOST) else 2
+    out = torch.empty(max(1, n.value) * width, dtype=torch.int32)
+    _check(lib().sta_plan_work_items(plan.handle, which, ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+                                     n.value, ctypes.byref(n), None), "sta_plan_work_items")
+    return out[: n.value * width].view(n.value, width), lone.value
 
 
 def sta_plan_q_tiles(plan: Plan, head: int):
