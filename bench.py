@@ -424,6 +424,10 @@ def run_ours(args):
     if rank == 0:
         peak_key = "bf16_tflops"
         peak = float(pk.get(peak_key, FALLBACK_PEAKS[peak_key]))
+        if bwd is not None:
+            # the backward's useful rate per GPU against the same measured bf16 peak
+            bwd["frac_of_peak"] = bwd["tflops_useful"] / world / peak
+            bwd["peak_source"] = f"{pk_kind} {peak_key}"
         achieved = flops / (ms * 1e-3) / 1e12
         traffic = profiled_traffic(wl.name)
         out = {
