@@ -12,7 +12,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("wl", [WORKLOADS["tiny"].with_(backward=True),
-                                Workload("graph_d128", 1, 2, 128, 6, 16, 24, (3, 8, 8), ((1, 1, 3), (2, 2, 2)),
+                                Workload("graph_d128", 1, 2, 128, 8, 8, 8, (4, 4, 4), ((1, 1, 1), (3, 3, 3)),
                                          backward=True)],
                          ids=lambda w: w.name)
 def test_forward_and_backward_replay_from_a_cuda_graph(wl):

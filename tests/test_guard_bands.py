@@ -38,7 +38,7 @@ def _bands_intact(whole, name):
 
 CASES = {
     "tiny_d64": WORKLOADS["tiny"].with_(backward=True),
-    "d128_partial_block": Workload("g1", 1, 2, 128, 6, 16, 24, (3, 8, 8), ((1, 1, 3), (2, 2, 2)), backward=True),
+    "d128_partial_block": Workload("g1", 1, 2, 128, 8, 8, 8, (4, 4, 4), ((1, 1, 1), (3, 3, 3)), backward=True),
     "d64_three_blocks_batch2": Workload("g2", 2, 1, 64, 12, 16, 16, (6, 8, 8), ((3, 3, 3),), backward=True),
     "d128_permute_fallback": Workload("g3", 1, 2, 128, 4, 12, 8, (2, 6, 4), ((3, 1, 2), (2, 2, 2)), backward=True),
 }
