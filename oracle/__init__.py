@@ -26,15 +26,24 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sta_oracle.c")
-_LIB = os.path.join(_HERE, "libsta_oracle.so")
+# STA_ORACLE_LIB names a prebuilt oracle library to load instead (the
+# mutation tests point it at copies of sta_oracle.c with a planted mistake)
+_LIB = os.environ.get("STA_ORACLE_LIB") or os.path.join(_HERE, "libsta_oracle.so")
 
 _lib = None
 
 
+def compile_command(src: str, out: str) -> list:
+    """gcc command that builds the oracle library `out` from `src`."""
+    return ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-o", out, src, "-lm"]
+
+
 def build(force: bool = False) -> str:
     """Compile sta_oracle.c into libsta_oracle.so (gcc, OpenMP, -O2)."""
+    if os.environ.get("STA_ORACLE_LIB"):
+        return _LIB
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"]
+        cmd = compile_command(_SRC, _LIB)
         subprocess.run(cmd, check=True)
     return _LIB
 
