@@ -171,8 +171,8 @@ sta_status sta_permute(sta_plan_t plan, const void *src, void *dst, int32_t inve
  * [batch][heads][N][head_dim]; lse is fp32 [batch][heads][N].  The softmax is
  * computed in fp32 with bf16 tensor-core products accumulated in fp32; o is
  * rounded to bf16 (nearest even).  `workspace` must hold at least fwd_bytes of
- * sta_plan_workspace_size; its first bytes carry the kernel status word that
- * STA_CALL_CHECK reads. */
+ * sta_plan_workspace_size (missing or smaller: STA_ERR_WORKSPACE); its first
+ * bytes carry the kernel status word that STA_CALL_CHECK reads. */
 sta_status sta_forward(sta_plan_t plan, const void *q, const void *k, const void *v, void *o,
                        float *lse, void *workspace, size_t workspace_bytes, void *stream,
                        uint32_t flags);
@@ -206,7 +206,8 @@ sta_status sta_forward_host(sta_plan_t plan, const void *q, const void *k, const
  * all sums running only over (query, key) pairs inside the window.  Inputs
  * q, k, v, o, dout bf16 and lse fp32 exactly as sta_forward produced them;
  * outputs dq, dk, dv bf16 of the same shape as q.  The plan must have been
- * created with STA_PROBLEM_BACKWARD; workspace >= bwd_bytes. */
+ * created with STA_PROBLEM_BACKWARD (else STA_ERR_INVALID_ARG); the workspace
+ * must hold bwd_bytes (missing or smaller: STA_ERR_WORKSPACE). */
 sta_status sta_backward(sta_plan_t plan, const void *q, const void *k, const void *v,
                         const void *o, const float *lse, const void *dout, void *dq, void *dk,
                         void *dv, void *workspace, size_t workspace_bytes, void *stream,
