@@ -142,6 +142,31 @@ class Problem:
                        bool(wl.backward if backward is None else backward), tiled, host_only, cta_pair)
 
 
+# Plans the garbage collector dropped without destroy(): (handle, device).
+# They are freed at the next safe point (see _free_dropped_plans).
+_DROPPED: list = []
+
+
+def _capturing() -> bool:
+    return torch.cuda.is_available() and torch.cuda.is_current_stream_capturing()
+
+
+def _free_dropped_plans():
+    """Free the plans the garbage collector dropped.  Kernels still queued may
+    read their tables, so each plan's device is synchronised first -- which is
+    not allowed while a stream is being captured into a CUDA graph, so then
+    they wait for the next call."""
+    if not _DROPPED or _capturing():
+        return
+    while _DROPPED:
+        handle, device = _DROPPED.pop()
+        try:
+            if device is not None:
+                torch.cuda.synchronize(device)
+        finally:
+            lib().sta_plan_destroy(handle)
+
+
 class Plan:
     """Owns an sta_plan_t.  Create with sta_plan_create()."""
 
@@ -167,16 +192,22 @@ class Plan:
     def destroy(self):
         """Free the plan.  Its device tables are read by every launch that uses
         it, so the plan's device is synchronised first: no such launch can
-        still be running when they are freed."""
+        still be running when they are freed.  Call it outside stream capture."""
         if self.handle is not None and self.handle.value:
             if self.device is not None:
                 torch.cuda.synchronize(self.device)
             _check(lib().sta_plan_destroy(self.handle), "sta_plan_destroy")
         self.handle = None
+        _free_dropped_plans()
 
     def __del__(self):
+        # The garbage collector runs anywhere -- inside a CUDA-graph capture
+        # too, where synchronising the device would break the capture -- so a
+        # dropped plan is only queued here and freed at the next safe point.
         try:
-            self.destroy()
+            if self.handle is not None and self.handle.value:
+                _DROPPED.append((self.handle, self.device))
+            self.handle = None
         except Exception:
             pass
 
@@ -190,6 +221,7 @@ class Plan:
 
 
 def sta_plan_create(problem: Problem) -> Plan:
+    _free_dropped_plans()
     cp, keep = problem._c()
     h = ctypes.c_void_p()
     _check(lib().sta_plan_create(ctypes.byref(cp), ctypes.byref(h)), "sta_plan_create")

@@ -219,6 +219,7 @@ def test_binding_passes_valid_device_buffers_through(monkeypatch):
         sta.sta_backward(plan, q, k, v, o, lse, do, dk=dev(torch.zeros(shape, dtype=torch.float32)),
                          workspace=ws, stream=0)
     assert len(rec.calls) == n  # none of them reached the library
+    plan.device = None  # it is a host-only plan again when it is freed
 
 
 def test_planner_reports_out_of_memory(tmp_path):
@@ -321,3 +322,21 @@ def test_autograd_and_plan_cache_marshalling(monkeypatch):
     assert len(sta._PLANS) == 2
     with pytest.raises(ValueError):
         sta.sliding_tile_attention(q, k, v, T, H, W, tile, [(3, 3, 3)] * 3)  # 3 windows, 2 heads
+
+
+def test_dropped_plans_are_freed_at_the_next_safe_point():
+    """A plan the garbage collector drops is not freed inside __del__ (which
+    may run during a CUDA-graph capture, where the device cannot be
+    synchronised) but queued, and freed by the next plan creation or destroy."""
+    import gc
+    sta._free_dropped_plans()
+    assert sta._DROPPED == []
+    plan = _create()
+    handle = plan.handle.value
+    del plan
+    gc.collect()
+    assert [h.value for h, _ in sta._DROPPED] == [handle]
+    other = _create()                      # a safe point: the dropped plan is freed
+    assert sta._DROPPED == []
+    other.destroy()
+    assert other.handle is None and sta._DROPPED == []
