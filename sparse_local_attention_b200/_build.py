@@ -32,6 +32,21 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
+def compile_command(src: str, obj: str) -> list:
+    """nvcc command that compiles one source of the library to an object."""
+    return [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
+
+
+def link_command(objs, out: str) -> list:
+    """nvcc command that links the objects into a shared library."""
+    return [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "--cudart", "shared", "-shared", "-o", out, *objs]
+
+
+def objects() -> dict:
+    """{source name: object path} of the last build."""
+    return {os.path.basename(s): os.path.join(PKG, "_build", os.path.basename(s) + ".o") for s in sources()}
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every source under csrc/ into sparse_local_attention_b200/libsta.so."""
     if not force and not _stale():
@@ -41,8 +56,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [_nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", src, "-o", obj]
-        return src, obj, subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, subprocess.run(compile_command(src, obj), capture_output=True, text=True)
 
     # the translation units are independent: compile them side by side
     with ThreadPoolExecutor(max_workers=max(1, min(len(SOURCES), os.cpu_count() or 1))) as ex:
@@ -55,8 +69,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             print(r.stderr)
         objs.append(obj)
     tmp = LIB + ".tmp"
-    cmd = [_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "--cudart", "shared", "-shared",
-           "-o", tmp, *objs]
+    cmd = link_command(objs, tmp)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")

@@ -53,7 +53,9 @@ _lib = None
 
 
 def library_path() -> str:
-    return _build.LIB
+    """libsta.so as built in-tree, or the build STA_LIBRARY names (the
+    planner's mutation tests load copies with a planted mistake that way)."""
+    return os.environ.get("STA_LIBRARY") or _build.LIB
 
 
 def lib() -> ctypes.CDLL:
@@ -61,9 +63,10 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(_build.LIB):
+    path = library_path()
+    if path == _build.LIB and not os.path.exists(path):
         _build.build()
-    L = ctypes.CDLL(_build.LIB)
+    L = ctypes.CDLL(path)
     vp, sz = ctypes.c_void_p, ctypes.c_size_t
     szp = ctypes.POINTER(ctypes.c_size_t)
     i32p = ctypes.POINTER(ctypes.c_int32)
