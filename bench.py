@@ -180,6 +180,85 @@ def call_stats(per_call_ms):
     return {"median": float(p50), "p10": float(p10), "p90": float(p90), "calls": len(per_call_ms)}
 
 
+def timed_leg(fn, warmup: int, steps: int, stream):
+    """warmup untimed calls, then steps calls timed with CUDA events on stream:
+    {"ms_per_call": mean, "per_call_ms": median / p10 / p90}."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms, per_call = timed_calls(fn, steps, stream)
+    return {"ms_per_call": ms, "per_call_ms": call_stats(per_call), "warmup": warmup, "steps": steps}
+
+
+def extra_legs(sta, peak: float, peak_source: str, stream, q, k, v, steps: int):
+    """The other workloads of the benchmark family, each timed on its own
+    inputs (resident in HBM, larger than L2) after 3 warm-up calls:
+      backward:     the fine-tuning workload's sta_backward, and its sta_forward;
+      perhead:      the per-head-window workload's sta_forward;
+      full_window:  the 720p latent with the window = the whole tile grid (dense
+                    attention through STA) beside the library's dense SDPA on
+                    the same tensors (q, k, v of the headline workload, which
+                    are the full-window workload's inputs: same shape, same seed)."""
+    def rate(flops, ms):
+        t = flops / (ms * 1e-3) / 1e12
+        return {"tflops_useful": t, "frac_of_peak": t / peak, "peak_source": peak_source}
+
+    legs = {}
+    # --- backward (fine-tuning workload)
+    wl = WORKLOADS["finetune"]
+    qf, kf, vf, dof = (x.cuda() for x in make_inputs(wl, with_dout=True))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=True))
+    of = torch.empty_like(qf)
+    lsef = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32, device="cuda")
+    fws, bws = plan.workspace(), plan.workspace(backward=True)
+    dq, dk, dv = torch.empty_like(qf), torch.empty_like(kf), torch.empty_like(vf)
+    sta.sta_forward(plan, qf, kf, vf, of, lsef, fws, stream, check=True)
+    sta.sta_backward(plan, qf, kf, vf, of, lsef, dof, dq, dk, dv, bws, stream, check=True)
+    fwd = timed_leg(lambda: sta.sta_forward(plan, qf, kf, vf, of, lsef, fws, stream), 3, steps, stream)
+    bwd = timed_leg(lambda: sta.sta_backward(plan, qf, kf, vf, of, lsef, dof, dq, dk, dv, bws, stream), 3, steps,
+                    stream)
+    legs["backward"] = {"workload": f"{wl.name}: {wl.description}", **bwd, **rate(wl.backward_flops(), bwd["ms_per_call"]),
+                        "useful_tflop_per_call": wl.backward_flops() / 1e12,
+                        "useful_flop_convention": "2.5 x forward (five GEMM-shaped products)",
+                        "kernels_per_call": plan.backward_launches,
+                        "forward": {**fwd, **rate(wl.forward_flops(), fwd["ms_per_call"]),
+                                    "useful_tflop_per_call": wl.forward_flops() / 1e12}}
+    plan.destroy()
+    del qf, kf, vf, dof, of, lsef, fws, bws, dq, dk, dv
+    # --- per-head windows
+    wl = WORKLOADS["dit720p_perhead"]
+    qp, kp, vp = (x.cuda() for x in make_inputs(wl))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl))
+    op = torch.empty_like(qp)
+    lsep = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32, device="cuda")
+    ws = plan.workspace()
+    sta.sta_forward(plan, qp, kp, vp, op, lsep, ws, stream, check=True)
+    fwd = timed_leg(lambda: sta.sta_forward(plan, qp, kp, vp, op, lsep, ws, stream), 3, steps, stream)
+    legs["perhead"] = {"workload": f"{wl.name}: {wl.description}", **fwd, **rate(wl.forward_flops(), fwd["ms_per_call"]),
+                       "useful_tflop_per_call": wl.forward_flops() / 1e12}
+    plan.destroy()
+    del qp, kp, vp, op, lsep, ws
+    # --- full window: dense attention through STA, beside the library's SDPA
+    wl = WORKLOADS["dit720p_full"]
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl))
+    o = torch.empty_like(q)
+    lse = torch.empty(wl.B, wl.Hh, wl.N, dtype=torch.float32, device="cuda")
+    ws = plan.workspace()
+    sta.sta_forward(plan, q, k, v, o, lse, ws, stream, check=True)
+    fwd = timed_leg(lambda: sta.sta_forward(plan, q, k, v, o, lse, ws, stream), 3, steps, stream)
+    sdpa = timed_leg(lambda: torch.nn.functional.scaled_dot_product_attention(q, k, v), 3, steps, stream)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    err = (o.float() - ref.float()).abs()
+    legs["full_window"] = {"workload": f"{wl.name}: {wl.description}", **fwd,
+                           **rate(wl.forward_flops(), fwd["ms_per_call"]),
+                           "useful_tflop_per_call": wl.forward_flops() / 1e12,
+                           "sdpa": {"impl": "torch.nn.functional.scaled_dot_product_attention (bf16)", **sdpa,
+                                    **rate(wl.forward_flops(), sdpa["ms_per_call"])},
+                           "sta_vs_sdpa_max_abs_diff": float(err.max()), "sta_vs_sdpa_mean_abs_diff": float(err.mean())}
+    plan.destroy()
+    return legs
+
+
 def timed_calls(fn, steps: int, stream):
     """Run fn steps times between CUDA events on stream, one event after each
     call; return (mean ms over the whole region, per-call ms)."""
@@ -420,6 +499,11 @@ def run_ours(args):
         tflops, dt, sample, cores, extra = time_oracle(wl, q_h, k_h, v_h, args.cpu_seconds)
         cpu = {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample, **extra}
 
+    legs = {}
+    if rank == 0 and world == 1 and args.workload == HEADLINE and not args.no_extra_legs:
+        peak_x = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        legs = extra_legs(sta, peak_x, f"{pk_kind} bf16_tflops", stream, q, k, v, max(10, min(args.steps, 20)))
+
     clocks = clk.summary()
     if rank == 0:
         peak_key = "bf16_tflops"
@@ -454,6 +538,10 @@ def run_ours(args):
             "backward": bwd,
             "permute": permute,
         }
+        if legs:
+            if out["backward"] is None:
+                out["backward"] = legs.pop("backward")
+            out.update(legs)
         print(json.dumps(out), flush=True)
     plan.destroy()
     if dist:
@@ -471,6 +559,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-legs", action="store_true",
+                    help="skip the backward / per-head / full-window records of the default run")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=384)
     ap.add_argument("--shard", default="problem", choices=["problem", "heads"],

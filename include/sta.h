@@ -27,6 +27,11 @@
  *     STA_CALL_CHECK is passed.
  *   - The caller owns every tensor and the workspace.  A plan owns its device
  *     tables and frees them in sta_plan_destroy.
+ *   - A plan's tables live on the device that was current when it was created,
+ *     and compute calls (sta_permute, sta_forward, sta_forward_host,
+ *     sta_backward, sta_backward_noalloc) enqueue on the calling thread's
+ *     current device: a call made while another device is current fails with
+ *     STA_ERR_INVALID_ARG and enqueues nothing.
  *   - A plan is immutable after creation and may be used from several streams
  *     at once as long as each concurrent call has its own workspace.
  *   - All argument checking happens on the host before any launch; a failing
@@ -63,14 +68,13 @@ typedef enum {
                                       with STA_ERR_INVALID_ARG.  For tooling and
                                       for inspecting lists on machines without
                                       a GPU. */
-#define STA_PROBLEM_CTA_PAIR 0x8u  /* run the forward pass on CTA pairs
-                                      (tcgen05 cta_group::2, M = 256 over two
-                                      SMs, each SM loading half of every K/V
-                                      chunk) where the geometry allows it: head
-                                      dim 128 and a tile volume that is a
-                                      multiple of 128.  Same results; by
-                                      default the one-CTA kernel runs, which is
-                                      faster on every shape measured so far. */
+#define STA_PROBLEM_DEVICE_CHECK_TEST 0x10u /* testing only: the plan is built
+                                      and uploaded as usual but records a
+                                      device number that is never current, so
+                                      every compute call on it fails the
+                                      device check (STA_ERR_INVALID_ARG) before
+                                      anything is enqueued.  Lets a machine
+                                      with one GPU test that check. */
 
 /* flags of sta_forward / sta_backward */
 #define STA_CALL_CHECK 0x1u /* synchronize `stream` after the launch and report
@@ -192,9 +196,8 @@ sta_status sta_plan_host_workspace_size(sta_plan_t plan, size_t *bytes);
  * ordered against `stream` with events (one cudaMemcpyAsync per tensor and
  * group).  The call returns after enqueueing; when `stream` reaches the end of
  * the call, o and lse are in host memory.  Copies overlap only for page-locked
- * host memory.  With tiles that are not TMA boxes of the raster tensor, or
- * with STA_PROBLEM_CTA_PAIR, the whole tensors are copied in, computed and
- * copied out in order.  Host buffers must stay valid and unchanged until
+ * host memory.  With tiles that are not TMA boxes of the raster tensor, the
+ * whole tensors are copied in, computed and copied out in order.  Host buffers must stay valid and unchanged until
  * `stream` has passed the call.  This call has no counterpart in the paper. */
 sta_status sta_forward_host(sta_plan_t plan, const void *q, const void *k, const void *v, void *o, float *lse,
                             void *workspace, size_t workspace_bytes, void *stream, uint32_t flags);
@@ -220,18 +223,23 @@ sta_status sta_backward(sta_plan_t plan, const void *q, const void *k, const voi
  * where the memory footprint must not change once set up -- and so cannot hand
  * over a workspace.  The temporaries go to a file-scope device array of 32 MiB
  * inside libsta.so instead; every GPU that loads the library holds that array
- * until the process exits.  Same arguments, results and flags as sta_backward,
- * minus the workspace.
+ * until the process exits.  Same arguments, results, flags and argument
+ * checks as sta_backward, minus the workspace.
  *   - Fails with STA_ERR_WORKSPACE when the plan's backward workspace
- *     (sta_plan_workspace_size, bwd_bytes) exceeds 32 MiB.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     (sta_plan_workspace_size, bwd_bytes) exceeds 32 MiB; the other argument
+ *     errors are those of sta_backward.  A failing call enqueues nothing.
+ *   - Uses the array of the plan's device, which must be the current one (as
+ *     for every compute call).  The first call on a device looks up the
+ *     array's device address (cudaGetSymbolAddress, with that device
+ *     current); make that first call before any stream capture.
  *   - Allocates nothing: no cudaMalloc / cudaFree, no allocating library call.
+ *     Enqueues exactly what sta_backward enqueues (with STA_CALL_CHECK, that
+ *     includes its status-word memset).
  *   - All calls share the one array, which keeps the previous call's contents;
- *     the status word is cleared on each call and the rest is rewritten before
- *     use.  Calls that overlap on the GPU (other streams, other host threads on
- *     the same device) race on it: order them. */
+ *     everything a call reads from it is written earlier in the same call (the
+ *     status word is cleared by STA_CALL_CHECK, which alone reads it).  Calls
+ *     that overlap on the GPU (other streams, other host threads on the same
+ *     device) race on it: order them. */
 sta_status sta_backward_noalloc(sta_plan_t plan, const void *q, const void *k, const void *v,
                                 const void *o, const float *lse, const void *dout, void *dq,
                                 void *dk, void *dv, void *stream, uint32_t flags);

@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsta.so")
-SOURCES = ["sta_api.cpp", "sta_permute.cu", "sta_fwd.cu", "sta_fwd_pair.cu", "sta_bwd.cu", "sta_noalloc.cu"]
+SOURCES = ["sta_api.cpp", "sta_permute.cu", "sta_fwd.cu", "sta_bwd.cu", "sta_noalloc.cu"]
 HEADERS = ["sm100_ptx.cuh", "sta_kernels.h", "sta_common.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
               "-Xcompiler", "-fPIC", "--cudart", "shared", "-Xptxas", "-v"]

@@ -41,8 +41,6 @@ struct sta_plan_s {
   int n_work_lone = 0;  // forward items with one query block, at the end of `work`
   int kv_mode = sta::kKvTiled;
   int piece_rows = 0, box_w = 0, box_h = 0, box_t = 0;
-  bool pair = false;  // forward runs on CTA pairs (sta_fwd_pair.cu)
-  int kh_box[3] = {0, 0, 0}, vh_box[3] = {0, 0, 0};  // raster boxes of 64 and 128 rows
   bool host_only = false;
   bool tiled = false;
   float scale = 0.f;
@@ -222,6 +220,20 @@ bool raster_box(const Geometry &g, int rows, int *bw, int *bh, int *bt) {
   return *bw <= 256 && *bh <= 256 && *bt <= 256;
 }
 
+// Compute calls enqueue on the calling thread's current device, and the plan's
+// tables live on the device that was current when it was created: a call made
+// while another device is current is refused before anything is enqueued.
+constexpr int kNoDevice = -2;
+
+sta_status check_device(const sta_plan_s *pl) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return STA_ERR_CUDA;
+  }
+  return dev == pl->device ? STA_OK : STA_ERR_INVALID_ARG;
+}
+
 sta_status finish_call(const sta_plan_s *pl, void *workspace, cudaStream_t stream, uint32_t flags) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return STA_ERR_CUDA;
@@ -236,7 +248,7 @@ sta_status finish_call(const sta_plan_s *pl, void *workspace, cudaStream_t strea
 }
 
 struct ForwardMaps {
-  CUtensorMap q, k, v, kh, vh;
+  CUtensorMap q, k, v;
   bool ok = false;
 };
 
@@ -249,10 +261,6 @@ ForwardMaps forward_maps(const sta_plan_s *pl, const void *qbase, const void *kb
                      make_map_raster(&m.v, vbase, pl))
                   : (make_map_tiled(&m.q, qbase, pl) && make_map_tiled(&m.k, kbase, pl) &&
                      make_map_tiled(&m.v, vbase, pl));
-  if (m.ok && pl->pair)
-    m.ok = raster5d ? (make_map_raster_box(&m.kh, kbase, pl, pl->kh_box[0], pl->kh_box[1], pl->kh_box[2], 2) &&
-                       make_map_raster_box(&m.vh, vbase, pl, pl->vh_box[0], pl->vh_box[1], pl->vh_box[2], 1))
-                    : (make_map_tiled_box(&m.kh, kbase, pl, 64, 2) && make_map_tiled_box(&m.vh, vbase, pl, 128, 1));
   return m;
 }
 
@@ -276,12 +284,28 @@ sta_status enqueue_forward(const sta_plan_s *pl, const ForwardMaps &maps, const 
   fp.box_w = pl->box_w, fp.box_h = pl->box_h, fp.box_t = pl->box_t;
   fp.box_panels = box_panels(pl);
   fp.oob_coord = raster5d ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
-  const cudaError_t e = pl->pair ? sta::launch_forward_pair(fp, maps.kh, maps.vh, pl->num_sms, stream)
-                                 : sta::launch_forward(fp, maps.q, maps.k, maps.v, pl->num_sms, stream);
+  const cudaError_t e = sta::launch_forward(fp, maps.q, maps.k, maps.v, pl->num_sms, stream);
   return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
 }
 
 }  // namespace
+
+namespace sta {
+
+// Every check of sta_backward except those of the workspace, in the order
+// sta_backward applies them; the last is the device check.
+sta_status check_backward_call(const sta_plan_s *pl, const void *const tensors[9], uint32_t flags) {
+  if (!pl || pl->host_only) return STA_ERR_INVALID_ARG;
+  for (int i = 0; i < 9; ++i)
+    if (!tensors[i]) return STA_ERR_INVALID_ARG;
+  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;  // plan built without STA_PROBLEM_BACKWARD
+  if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  for (int i = 0; i < 9; ++i)
+    if (!aligned16(tensors[i])) return STA_ERR_ALIGNMENT;
+  return check_device(pl);
+}
+
+}  // namespace sta
 
 extern "C" {
 
@@ -304,7 +328,7 @@ void sta_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
 
 sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
   if (!prob || !out || !prob->window) return STA_ERR_INVALID_ARG;
-  const uint32_t known = STA_PROBLEM_BACKWARD | STA_PROBLEM_TILED | STA_PROBLEM_HOST_ONLY | STA_PROBLEM_CTA_PAIR;
+  const uint32_t known = STA_PROBLEM_BACKWARD | STA_PROBLEM_TILED | STA_PROBLEM_HOST_ONLY | STA_PROBLEM_DEVICE_CHECK_TEST;
   if (prob->flags & ~known) return STA_ERR_INVALID_ARG;
   if (prob->batch < 1 || prob->heads < 1 || prob->T < 1 || prob->H < 1 || prob->W < 1 || prob->tile_t < 1 ||
       prob->tile_h < 1 || prob->tile_w < 1)
@@ -509,17 +533,6 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
     pl->kv_mode = sta::kKvTiled;  // permute K and V into the workspace first
   }
 
-  // CTA-pair forward (on request): head dim 128, whole 128-row chunks inside a
-  // tile, and (for raster inputs read in place) 64- and 128-row runs that are boxes.
-  if ((prob->flags & STA_PROBLEM_CTA_PAIR) && g.d == 128 && g.tau % 128 == 0) {
-    if (pl->kv_mode == sta::kKvTiled) {
-      pl->pair = true;
-    } else {
-      pl->pair = raster_box(g, 64, &pl->kh_box[0], &pl->kh_box[1], &pl->kh_box[2]) &&
-                 raster_box(g, 128, &pl->vh_box[0], &pl->vh_box[1], &pl->vh_box[2]);
-    }
-  }
-
   if (!pl->host_only) {
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -534,7 +547,8 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
       delete pl;
       return STA_ERR_UNSUPPORTED;
     }
-    pl->device = dev;
+    // (a plan made for the device-check test records a device that is never current)
+    pl->device = (prob->flags & STA_PROBLEM_DEVICE_CHECK_TEST) ? kNoDevice : dev;
     std::vector<int32_t> cnt(pl->count);
     if (!upload(&pl->d_kv_list, pl->kv_list) || !upload(&pl->d_count, cnt) || !upload(&pl->d_work, pl->work) ||
         !upload(&pl->d_work_host, pl->work_host) ||
@@ -602,8 +616,7 @@ sta_status sta_plan_launches(sta_plan_t pl, int32_t *forward, int32_t *backward)
   const bool gather = !pl->tiled && pl->kv_mode != sta::kKvRaster;  // permute Q, K, V (and dO) first
   if (forward) {
     int f = gather ? 3 : 0;
-    if (pl->pair) f += n_work > 0 ? 1 : 0;
-    else f += (n_work - pl->n_work_lone > 0 ? 1 : 0) + (pl->n_work_lone > 0 ? 1 : 0);
+    f += (n_work - pl->n_work_lone > 0 ? 1 : 0) + (pl->n_work_lone > 0 ? 1 : 0);
     *forward = f;
   }
   if (backward) {
@@ -652,6 +665,7 @@ sta_status sta_permute(sta_plan_t pl, const void *src, void *dst, int32_t invers
   const size_t bytes = tensor_bytes(pl);
   const char *s = static_cast<const char *>(src), *d = static_cast<const char *>(dst);
   if (s < d + bytes && d < s + bytes) return STA_ERR_INVALID_ARG;
+  if (const sta_status dev_st = check_device(pl)) return dev_st;
   sta::PermuteParams pp{};
   pp.g = pl->g;
   pp.src = src;
@@ -670,6 +684,7 @@ sta_status sta_forward(sta_plan_t pl, const void *q, const void *k, const void *
     return STA_ERR_ALIGNMENT;
   if (!workspace || ws_bytes < fwd_workspace(pl)) return STA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return STA_ERR_ALIGNMENT;
+  if (const sta_status dev_st = check_device(pl)) return dev_st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(ws);
@@ -712,6 +727,7 @@ sta_status sta_forward_host(sta_plan_t pl, const void *q, const void *k, const v
   if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < host_workspace(pl)) return STA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return STA_ERR_ALIGNMENT;
+  if (const sta_status dev_st = check_device(pl)) return dev_st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   const size_t tb = tensor_bytes(pl), tb_r = round256(tb);
   char *ws = static_cast<char *>(workspace);
@@ -721,7 +737,7 @@ sta_status sta_forward_host(sta_plan_t pl, const void *q, const void *k, const v
   const size_t fwd_bytes = fwd_workspace(pl);
   const bool gather = !pl->tiled && pl->kv_mode != sta::kKvRaster;
 
-  if (gather || pl->pair) {
+  if (gather) {
     // no slice pipeline on these paths: whole tensors in, one sta_forward, whole outputs out
     if ((flags & STA_CALL_CHECK) && cudaMemsetAsync(ws_fwd, 0, sizeof(int), stream) != cudaSuccess)
       return STA_ERR_CUDA;
@@ -795,14 +811,11 @@ sta_status sta_forward_host(sta_plan_t pl, const void *q, const void *k, const v
 sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void *v, const void *o,
                         const float *lse, const void *dout, void *dq, void *dk, void *dv, void *workspace,
                         size_t ws_bytes, void *stream_, uint32_t flags) {
-  if (!pl || !q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || pl->host_only)
-    return STA_ERR_INVALID_ARG;
-  if (pl->inv_off.empty()) return STA_ERR_INVALID_ARG;  // plan built without STA_PROBLEM_BACKWARD
-  if (flags & ~STA_CALL_CHECK) return STA_ERR_INVALID_ARG;
+  const void *tensors[9] = {q, k, v, o, lse, dout, dq, dk, dv};
+  sta_status st = sta::check_backward_call(pl, tensors, flags);
+  if (st != STA_OK) return st;
   if (!workspace || ws_bytes < bwd_workspace(pl)) return STA_ERR_WORKSPACE;
-  const void *ptrs[10] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
-  for (const void *ptr : ptrs)
-    if (!aligned16(ptr)) return STA_ERR_ALIGNMENT;
+  if (!aligned16(workspace)) return STA_ERR_ALIGNMENT;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);
   int *status = reinterpret_cast<int *>(ws);

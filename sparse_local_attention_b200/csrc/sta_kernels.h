@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "../../include/sta.h"
+
 namespace sta {
 
 // Status codes the kernels write into the workspace status word.
@@ -93,10 +95,10 @@ struct PermuteParams {
 
 cudaError_t launch_forward(const FwdParams &p, const CUtensorMap &tmap_q, const CUtensorMap &tmap_k,
                            const CUtensorMap &tmap_v, int num_sms, cudaStream_t stream);
-// Forward on CTA pairs (head dim 128, tile volume a multiple of 128): K halves
-// (64 keys, both panels) and V halves (128 keys, one panel) per CTA.
-cudaError_t launch_forward_pair(const FwdParams &p, const CUtensorMap &tmap_k_half, const CUtensorMap &tmap_v_half,
-                                int num_sms, cudaStream_t stream);
+// The argument checks of sta_backward other than those of the workspace
+// (null, host-only or forward-only plan, flags, alignment, current device).
+sta_status check_backward_call(const sta_plan_s *plan, const void *const tensors[9], uint32_t flags);
+
 cudaError_t launch_permute(const PermuteParams &p, int num_sms, cudaStream_t stream);
 // Backward: preprocess (D, LSE*log2 e), dK/dV (key-block major) and dQ
 // (query-block major), enqueued in that order on `stream`.

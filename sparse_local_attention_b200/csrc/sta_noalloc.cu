@@ -13,16 +13,18 @@
 //
 // The array has a fixed size (kNoallocScratchBytes).  Every GPU that loads
 // this library holds it in device memory until the process exits.  All calls
-// share it and it keeps whatever the last call left there: the status word is
-// cleared on every call, everything else is fully written before it is read.
-// Calls whose execution overlaps on the GPU (different streams, or different
-// host threads on one device) race on the array and give wrong results; the
-// caller must order them.
+// share it and it keeps whatever the last call left there: everything a call
+// reads from it is written earlier in the same call (the status word is
+// cleared by STA_CALL_CHECK, the only reader of it).  Calls whose execution
+// overlaps on the GPU (different streams, or different host threads on one
+// device) race on the array and give wrong results; the caller must order
+// them.
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "../../include/sta.h"
+#include "sta_kernels.h"
 
 namespace {
 
@@ -37,6 +39,9 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 std::mutex g_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
+// The device address of the array on the current device (looked up once per
+// device).  Called after the device check, so the current device is the
+// plan's.
 sta_status scratch_for_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -68,12 +73,13 @@ sta_status sta_backward_noalloc(sta_plan_t plan, const void *q, const void *k, c
   sta_status st = sta_plan_workspace_size(plan, nullptr, &need);
   if (st != STA_OK) return st;
   if (need > kNoallocScratchBytes) return STA_ERR_WORKSPACE;
+  // every other check of sta_backward, before the array is looked up
+  const void *tensors[9] = {q, k, v, o, lse, dout, dq, dk, dv};
+  st = sta::check_backward_call(plan, tensors, flags);
+  if (st != STA_OK) return st;
   void *scratch = nullptr;
   st = scratch_for_current_device(&scratch);
   if (st != STA_OK) return st;
-  // The status word must start at zero for STA_CALL_CHECK to mean anything;
-  // clear it on every call (an enqueued memset, not an allocation).
-  if (cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) return STA_ERR_CUDA;
   return sta_backward(plan, q, k, v, o, lse, dout, dq, dk, dv, scratch, kNoallocScratchBytes, stream, flags);
 }
 

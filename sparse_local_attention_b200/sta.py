@@ -7,6 +7,7 @@ call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -25,7 +26,7 @@ STATUS_NAMES = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_SHAPE", 3: "S
 STA_PROBLEM_BACKWARD = 0x1
 STA_PROBLEM_TILED = 0x2
 STA_PROBLEM_HOST_ONLY = 0x4
-STA_PROBLEM_CTA_PAIR = 0x8
+STA_PROBLEM_DEVICE_CHECK_TEST = 0x10
 STA_CALL_CHECK = 0x1
 
 EXPORTED = ["sta_plan_create", "sta_plan_destroy", "sta_plan_workspace_size", "sta_plan_kv_tiles",
@@ -128,21 +129,21 @@ class Problem:
     backward: bool = False
     tiled: bool = False
     host_only: bool = False
-    cta_pair: bool = False
+    extra_flags: int = 0  # other STA_PROBLEM_* bits (the device-check test flag)
 
     def _c(self):
         flat = [int(x) for w in self.windows for x in w]
         arr = (ctypes.c_int32 * max(1, len(flat)))(*flat)
         flags = ((STA_PROBLEM_BACKWARD if self.backward else 0) | (STA_PROBLEM_TILED if self.tiled else 0)
-                 | (STA_PROBLEM_HOST_ONLY if self.host_only else 0) | (STA_PROBLEM_CTA_PAIR if self.cta_pair else 0))
+                 | (STA_PROBLEM_HOST_ONLY if self.host_only else 0) | int(self.extra_flags))
         p = _Problem(self.batch, self.heads, self.head_dim, self.T, self.H, self.W, *self.tile,
                      ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), float(self.scale), flags)
         return p, arr
 
     @staticmethod
-    def from_workload(wl, backward=None, tiled=False, host_only=False, scale=0.0, cta_pair=False) -> "Problem":
+    def from_workload(wl, backward=None, tiled=False, host_only=False, scale=0.0) -> "Problem":
         return Problem(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows), scale,
-                       bool(wl.backward if backward is None else backward), tiled, host_only, cta_pair)
+                       bool(wl.backward if backward is None else backward), tiled, host_only)
 
 
 # Plans the garbage collector dropped without destroy(): (handle, device).
@@ -308,13 +309,25 @@ def _nbytes(t: torch.Tensor) -> int:
     return t.numel() * t.element_size()
 
 
+def _on_plan_device(plan: Plan):
+    """Context in which a compute call runs: the plan's device made current.
+    The library enqueues on the current device (and refuses a call made while
+    another device is current), and the default stream of a call is the
+    current stream of that device."""
+    if plan.device is None:
+        return contextlib.nullcontext()
+    return torch.cuda.device(plan.device)
+
+
 def sta_permute(plan: Plan, src: torch.Tensor, dst: Optional[torch.Tensor] = None, inverse: bool = False,
                 stream=None) -> torch.Tensor:
     _expect(src, "src", _shape(plan), torch.bfloat16, plan.device)
     if dst is None:
         dst = torch.empty_like(src)
     _expect(dst, "dst", _shape(plan), torch.bfloat16, plan.device)
-    _check(lib().sta_permute(plan.handle, _ptr(src), _ptr(dst), 1 if inverse else 0, _stream(stream)), "sta_permute")
+    with _on_plan_device(plan):
+        _check(lib().sta_permute(plan.handle, _ptr(src), _ptr(dst), 1 if inverse else 0, _stream(stream)),
+               "sta_permute")
     return dst
 
 
@@ -332,8 +345,9 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     if lse is not None:
         _expect(lse, "lse", shape[:3], torch.float32, dev)
     workspace = _workspace(plan, workspace)
-    st = lib().sta_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
-                           _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
+    with _on_plan_device(plan):
+        st = lib().sta_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                               _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_forward")
     return o, lse
 
@@ -361,8 +375,9 @@ def sta_forward_host(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     if lse is not None:
         _expect_host(lse, "lse", shape[:3], torch.float32)
     workspace = _workspace(plan, workspace, host=True)
-    st = lib().sta_forward_host(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
-                                _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
+    with _on_plan_device(plan):
+        st = lib().sta_forward_host(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace),
+                                    _nbytes(workspace), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_forward_host")
     return o, lse
 
@@ -379,9 +394,10 @@ def sta_backward(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv=None, w
     for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _expect(t, nm, shape, torch.bfloat16, dev)
     workspace = _workspace(plan, workspace, backward=True)
-    st = lib().sta_backward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                            _ptr(dk), _ptr(dv), _ptr(workspace), _nbytes(workspace), _stream(stream),
-                            STA_CALL_CHECK if check else 0)
+    with _on_plan_device(plan):
+        st = lib().sta_backward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                                _ptr(dk), _ptr(dv), _ptr(workspace), _nbytes(workspace), _stream(stream),
+                                STA_CALL_CHECK if check else 0)
     _check(st, "sta_backward")
     return dq, dk, dv
 
@@ -400,8 +416,9 @@ def sta_backward_noalloc(plan: Plan, q, k, v, o, lse, dout, dq=None, dk=None, dv
     dv = torch.empty_like(v) if dv is None else dv
     for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _expect(t, nm, shape, torch.bfloat16, dev)
-    st = lib().sta_backward_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
-                                    _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream), STA_CALL_CHECK if check else 0)
+    with _on_plan_device(plan):
+        st = lib().sta_backward_noalloc(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                        _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream), STA_CALL_CHECK if check else 0)
     _check(st, "sta_backward_noalloc")
     return dq, dk, dv
 
@@ -440,7 +457,7 @@ def cached_plan(problem: Problem) -> Plan:
     still hold it for its backward)."""
     key = (problem.batch, problem.heads, problem.head_dim, problem.T, problem.H, problem.W, tuple(problem.tile),
            tuple(tuple(int(x) for x in w) for w in problem.windows), float(problem.scale), problem.backward,
-           problem.tiled, problem.cta_pair, torch.cuda.current_device())
+           problem.tiled, problem.extra_flags, torch.cuda.current_device())
     with _PLANS_LOCK:
         plan = _PLANS.get(key)
         if plan is not None:

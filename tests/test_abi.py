@@ -155,16 +155,42 @@ class _OnCuda1(_OnCuda0):
 
 
 class _RecordingLib:
-    """Stands in for libsta.so: records each call's arguments, returns STA_OK."""
+    """Stands in for libsta.so: records each call's arguments, returns STA_OK;
+    `devices` records the device current (under _FakeDevices) at each call."""
 
-    def __init__(self):
+    def __init__(self, devices=None):
         self.calls = []
+        self.devices = []
+        self.current = devices
 
     def __getattr__(self, name):
         def call(*args):
             self.calls.append((name, args))
+            self.devices.append(self.current.now if self.current is not None else None)
             return 0
         return call
+
+
+class _FakeDevices:
+    """Stands in for torch.cuda.device / current_device on a machine without
+    a GPU: a device context that only records which device it made current."""
+
+    def __init__(self, start=0):
+        self.now = start
+
+    def current_device(self):
+        return self.now
+
+    def device(self, index):
+        fake = self
+
+        class _Ctx:
+            def __enter__(self):
+                self.prev, fake.now = fake.now, index
+
+            def __exit__(self, *exc):
+                fake.now = self.prev
+        return _Ctx()
 
 
 def test_binding_passes_valid_device_buffers_through(monkeypatch):
@@ -178,7 +204,9 @@ def test_binding_passes_valid_device_buffers_through(monkeypatch):
     q, k, v, o, do = (dev(torch.zeros(shape, dtype=torch.bfloat16)) for _ in range(5))
     lse = dev(torch.zeros(shape[:3], dtype=torch.float32))
     ws = dev(torch.zeros(100, dtype=torch.float32))  # 400 bytes
-    rec = _RecordingLib()
+    fake = _FakeDevices()
+    monkeypatch.setattr(torch.cuda, "device", fake.device)
+    rec = _RecordingLib(fake)
     monkeypatch.setattr(sta, "lib", lambda: rec)
 
     sta.sta_forward(plan, q, k, v, o, lse, ws, stream=0, check=True)
@@ -281,6 +309,7 @@ def test_autograd_and_plan_cache_marshalling(monkeypatch):
     monkeypatch.setattr(sta, "lib", lambda: rec)
     monkeypatch.setattr(sta, "_PLANS", OrderedDict())
     monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(torch.cuda, "device", _FakeDevices().device)
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: None)
     monkeypatch.setattr(sta, "_stream", lambda stream: ctypes.c_void_p(0))
 
@@ -340,3 +369,46 @@ def test_dropped_plans_are_freed_at_the_next_safe_point():
     assert sta._DROPPED == []
     other.destroy()
     assert other.handle is None and sta._DROPPED == []
+
+
+def test_binding_makes_the_plan_device_current_for_each_call(monkeypatch):
+    """The library enqueues on the current device and refuses a call made
+    while another device is current, so the binding makes the plan's device
+    current around every compute call (and only there): a plan of cuda:1 used
+    while cuda:0 is current still runs on cuda:1."""
+    plan = _create(backward=True)
+    plan.device = 1  # as if the tables had been uploaded to cuda:1
+    shape = (1, 1, 4 * 8 * 8, 64)
+    dev = lambda t: t.as_subclass(_OnCuda1)
+    q, o, do = (dev(torch.zeros(shape, dtype=torch.bfloat16)) for _ in range(3))
+    lse = dev(torch.zeros(shape[:3], dtype=torch.float32))
+    ws = dev(torch.zeros(100, dtype=torch.float32))
+    fake = _FakeDevices(start=0)
+    monkeypatch.setattr(torch.cuda, "device", fake.device)
+    rec = _RecordingLib(fake)
+    monkeypatch.setattr(sta, "lib", lambda: rec)
+    sta.sta_forward(plan, q, q, q, o, lse, ws, stream=0)
+    sta.sta_backward(plan, q, q, q, o, lse, do, q.clone(), q.clone(), q.clone(), workspace=ws, stream=0)
+    sta.sta_backward_noalloc(plan, q, q, q, o, lse, do, q.clone(), q.clone(), q.clone(), stream=0)
+    sta.sta_permute(plan, q, o, stream=0)
+    qh = torch.zeros(shape, dtype=torch.bfloat16)
+    sta.sta_forward_host(plan, qh, qh, qh, workspace=ws, stream=0)
+    names = [c[0] for c in rec.calls]
+    assert names == ["sta_forward", "sta_backward", "sta_backward_noalloc", "sta_permute", "sta_forward_host"]
+    assert rec.devices == [1] * 5
+    assert fake.now == 0  # the caller's device is current again afterwards
+    plan.device = None
+
+
+def test_noalloc_checks_its_arguments_before_anything_else():
+    """sta_backward_noalloc applies sta_backward's argument checks before it
+    looks up its scratch array or enqueues anything: a host-only plan is an
+    invalid argument (not a CUDA error), as are null tensors and unknown
+    flags; misaligned tensors are an alignment error."""
+    plan = _create(backward=True)
+    L = sta.lib()
+    ok = [ctypes.c_void_p(256 * (i + 1)) for i in range(9)]
+    assert L.sta_backward_noalloc(plan.handle, *ok, None, 0) == 1           # host-only plan
+    fwd_only = _create()
+    assert L.sta_backward_noalloc(fwd_only.handle, *ok, None, 0) == 1       # host-only, no backward tables
+    assert L.sta_backward_noalloc(None, *ok, None, 0) == 1

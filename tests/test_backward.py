@@ -93,25 +93,28 @@ def test_backward_is_deterministic():
 
 def test_finetune_sampled_rows():
     """The fine-tuning workload (2x16 heads, 16x64x64, tile 4x8x8, window
-    3x5x5): dQ on sampled rows of 64 query tiles for 4 slices, dK/dV on
-    sampled rows of 64 key tiles (8 corners + 56 seeded) for the same 4
-    slices."""
+    3x5x5): dQ on 16 rows (first, last and 14 seeded) of each of 64 query
+    tiles (8 corners + 56 seeded) for all 32 (batch, head) slices; dK/dV on 4
+    rows of each of 64 key tiles for 4 seeded slices (each of those needs the
+    oracle's LSE and D for almost every query of the slice)."""
     wl = WORKLOADS["finetune"]
     q, k, v, do = make_inputs(wl, with_dout=True)
     _, _, (dq, dk, dv) = run_fwd_bwd(wl, q, k, v, do)
     g = geom_of(wl)
     rng = np.random.default_rng(0)
-    slices = [0, 17, 2 * wl.Hh - 1, 9]
     qtiles = tiles_sample(wl, 64, seed=0)
-    for bh in slices:
+    assert len(qtiles) == 64
+    dq_host = dq.cpu()
+    for bh in range(wl.B * wl.Hh):
         rows = []
         for t in qtiles:
             toks = tile_tokens(wl, t)
-            rows += [toks[0], toks[-1]] + list(rng.choice(toks, 4, replace=False))
+            rows += [toks[0], toks[-1]] + list(rng.choice(toks[1:-1], 14, replace=False))
         rows = np.array(sorted(set(rows)))
         b, h = divmod(bh, wl.Hh)
         rdq, _, _ = oracle.backward(g, q, k, v, do, bh, q_rows=rows, k_rows=np.zeros(0, dtype=np.int64))
-        compare(f"dq[{bh}]", dq[b, h, torch.as_tensor(rows)].double().cpu().numpy(), rdq)
+        compare(f"dq[{bh}]", dq_host[b, h, torch.as_tensor(rows)].double().numpy(), rdq)
+    slices = [0, 17, 2 * wl.Hh - 1, 9]
     ktiles = tiles_sample(wl, 64, seed=1)
     for bh in slices:
         rows = []

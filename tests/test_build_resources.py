@@ -15,7 +15,7 @@ import pytest
 
 from sparse_local_attention_b200 import _build
 
-KERNELS = ("sta_fwd_kernel", "sta_fwd_pair_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel",
+KERNELS = ("sta_fwd_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel",
            "bwd_dkdv_kernel")
 
 
@@ -58,12 +58,11 @@ def test_kernel_register_budgets(tmp_path):
     res = _resources(tmp_path)
     for k in KERNELS:
         assert k in res, f"{k}: no ptxas report"
-    for k in ("sta_fwd_kernel", "sta_fwd_pair_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel"):
+    for k in ("sta_fwd_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel"):
         for mangled, regs, spill in res[k]:
             assert spill == 0, f"{k} ({mangled}) spills {spill} bytes"
-    for k, cap in (("sta_fwd_kernel", 168), ("sta_fwd_pair_kernel", 168)):
-        for mangled, regs, spill in res[k]:
-            assert regs <= cap, (k, mangled, regs)
+    for mangled, regs, spill in res["sta_fwd_kernel"]:
+        assert regs <= 168, (mangled, regs)
     for mangled, regs, spill in res["bwd_dkdv_kernel"] + res["bwd_dq_kernel"]:
         # head dim 64 runs 576 threads (96 registers), head dim 128 320 (168)
         cap = 96 if "ILi64E" in mangled else 168

@@ -24,8 +24,8 @@ def geom_of(wl: Workload) -> Geometry:
     return Geometry(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, tuple(wl.tile), tuple(wl.windows))
 
 
-def run_gpu(wl: Workload, q, k, v, tiled=False, cta_pair=False):
-    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, tiled=tiled, cta_pair=cta_pair))
+def run_gpu(wl: Workload, q, k, v, tiled=False):
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, tiled=tiled))
     qd, kd, vd = (x.cuda() for x in (q, k, v))
     o, lse = sta.sta_forward(plan, qd, kd, vd, check=True)
     torch.cuda.synchronize()
@@ -79,11 +79,11 @@ SMALL = {
     # windows that are distinct for some tiles: their last blocks stay lone (split across warpgroups)
     "d128_lone_blocks_split": Workload("l", 1, 2, 128, 4, 8, 32, (2, 8, 8), ((1, 1, 2), (1, 1, 3))),
     "d64_lone_block_odd_chunks": Workload("m", 2, 1, 64, 2, 8, 40, (2, 8, 8), ((1, 1, 3),)),
-    # tile volumes that are multiples of 128 (also run on CTA pairs below)
-    "d128_pair_tau128_one_block": Workload("h", 1, 2, 128, 4, 16, 16, (2, 8, 8), ((3, 3, 3), (1, 2, 2))),
-    "d128_pair_tau256": Workload("i", 2, 1, 128, 8, 16, 24, (4, 8, 8), ((2, 3, 3),)),
-    "d128_pair_tau384_odd_blocks": Workload("j", 1, 2, 128, 12, 16, 16, (6, 8, 8), ((3, 3, 3), (1, 1, 1))),
-    "d128_pair_tau256_big_window": Workload("k", 1, 1, 128, 8, 24, 24, (4, 8, 8), ((5, 5, 5),)),
+    # tile volumes that are multiples of 128
+    "d128_tau128_one_block": Workload("h", 1, 2, 128, 4, 16, 16, (2, 8, 8), ((3, 3, 3), (1, 2, 2))),
+    "d128_tau256": Workload("i", 2, 1, 128, 8, 16, 24, (4, 8, 8), ((2, 3, 3),)),
+    "d128_tau384_odd_blocks": Workload("j", 1, 2, 128, 12, 16, 16, (6, 8, 8), ((3, 3, 3), (1, 1, 1))),
+    "d128_tau256_big_window": Workload("k", 1, 1, 128, 8, 24, 24, (4, 8, 8), ((5, 5, 5),)),
 }
 
 
@@ -96,33 +96,13 @@ def test_forward_small_all_rows(name):
     compare_rows(wl, o, lse, q, k, v, rows)
 
 
-PAIR_CASES = [n for n in SMALL if n.startswith("d128_pair")]
-
-
-@pytest.mark.parametrize("name", PAIR_CASES)
-def test_forward_cta_pair_all_rows(name):
-    """The CTA-pair kernel (STA_PROBLEM_CTA_PAIR) against the oracle."""
-    wl = SMALL[name]
-    q, k, v = make_inputs(wl, seed=1)
-    o, lse, _ = run_gpu(wl, q, k, v, cta_pair=True)
-    compare_rows(wl, o, lse, q, k, v, np.arange(wl.B * wl.Hh * wl.N))
-
-
-def test_forward_cta_pair_dit720p_sampled():
-    wl = WORKLOADS["dit720p"]
-    q, k, v = make_inputs(wl)
-    o, lse, _ = run_gpu(wl, q, k, v, cta_pair=True)
-    compare_rows(wl, o, lse, q, k, v, sampled_rows(wl, 32, 6))
-
-
-@pytest.mark.parametrize("name,cta_pair", [("d128_tau48_boxes_of_16", False), ("d128_pair_tau384_odd_blocks", False),
-                                           ("d128_pair_tau384_odd_blocks", True)])
-def test_forward_tiled_layout_matches_raster(name, cta_pair):
+@pytest.mark.parametrize("name", ["d128_tau48_boxes_of_16", "d128_tau384_odd_blocks"])
+def test_forward_tiled_layout_matches_raster(name):
     wl = SMALL[name]
     q, k, v = make_inputs(wl, seed=2)
-    o, lse, plan = run_gpu(wl, q, k, v, cta_pair=cta_pair)
+    o, lse, plan = run_gpu(wl, q, k, v)
     qt, kt, vt = (sta.sta_permute(plan, x.cuda()) for x in (q, k, v))
-    plan_t = sta.sta_plan_create(sta.Problem.from_workload(wl, tiled=True, cta_pair=cta_pair))
+    plan_t = sta.sta_plan_create(sta.Problem.from_workload(wl, tiled=True))
     o_t, lse_t = sta.sta_forward(plan_t, qt, kt, vt, check=True)
     o_back = sta.sta_permute(plan, o_t, inverse=True)
     torch.cuda.synchronize()
@@ -178,13 +158,31 @@ def test_one_hot_tile_coordinates_full_scale(name):
 
 
 # ----------------------------------------------------------------- sampled oracle on the large workloads
-@pytest.mark.parametrize("name,rows_per_tile", [("dit720p", 12), ("dit720p_perhead", 8), ("finetune", 12),
-                                                ("dit720p_full", 2)])
-def test_forward_large_sampled(name, rows_per_tile):
+# Whole query tiles: the 8 corner tiles of the grid (where the window is
+# shifted inward) and 56 seeded others, every row of each.  Heads: every head
+# of the 720p and fine-tuning workloads; on the per-head workload two heads of
+# each window class (1x3x3, 3x3x5, 5x5x5).  The full-window workload (115200
+# keys per row) is compared with the library's dense attention on every row
+# and with the oracle on sampled rows of the same tiles.
+LARGE = {
+    # name: (rows per tile or None for all, heads or None for all)
+    "dit720p": (None, None),
+    "dit720p_perhead": (None, (0, 7, 8, 15, 16, 23)),
+    "finetune": (None, None),
+    "dit720p_full": (2, None),
+}
+
+
+@pytest.mark.parametrize("name", list(LARGE))
+def test_forward_large_sampled(name):
     wl = WORKLOADS[name]
+    rows_per_tile, heads = LARGE[name]
     q, k, v = make_inputs(wl)
     o, lse, _ = run_gpu(wl, q, k, v)
-    rows = sampled_rows(wl, 64, rows_per_tile)
+    bh_list = None if heads is None else [b * wl.Hh + h for b in range(wl.B) for h in heads]
+    rows = sampled_rows(wl, 64, rows_per_tile, bh_list=bh_list)
+    if rows_per_tile is None:
+        assert len(rows) == 64 * wl.tile_volume * (wl.B * wl.Hh if heads is None else len(bh_list))
     compare_rows(wl, o, lse, q, k, v, rows)
     if name == "dit720p_full":
         # the whole output against the library's dense attention on the GPU
@@ -201,17 +199,17 @@ def test_tiny_workload_full_oracle():
 
 
 # ----------------------------------------------------------------- host tensors (sta_forward_host)
-@pytest.mark.parametrize("name,pinned,cta_pair", [
-    ("d128_pair_tau384_odd_blocks", True, False),   # 2 slices, pairs and lone blocks
-    ("d64_tau192_partial_block", True, False),      # batch 2: 4 slices in 4 groups
-    ("d128_permute_fallback", True, False),         # gather path: copied whole, not pipelined
-    ("d128_pair_tau256", True, True),               # CTA-pair kernel: not pipelined
-    ("tiny_workload", False, False),                # pageable host memory
+@pytest.mark.parametrize("name,pinned", [
+    ("d128_tau384_odd_blocks", True),     # 2 slices, pairs and lone blocks
+    ("d64_tau192_partial_block", True),   # batch 2: 4 slices in 4 groups
+    ("d128_permute_fallback", True),      # gather path: copied whole, not pipelined
+    ("d128_tau256", True),                # two query blocks per tile
+    ("tiny_workload", False),             # pageable host memory
 ])
-def test_forward_host_equals_device_call(name, pinned, cta_pair):
+def test_forward_host_equals_device_call(name, pinned):
     wl = SMALL[name]
     q, k, v = make_inputs(wl, seed=4)
-    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False, cta_pair=cta_pair))
+    plan = sta.sta_plan_create(sta.Problem.from_workload(wl, backward=False))
     _host_vs_device(plan, q, k, v, pinned)
 
 

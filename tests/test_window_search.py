@@ -1,5 +1,5 @@
 """Per-head window search: the selection rule on the host (fake forward), and
-the search through sta_forward on the GPU against dense attention."""
+the search through sta_forward on the GPU against the fp64 oracle."""
 import pytest
 import torch
 
@@ -60,22 +60,41 @@ def test_clamped_keys_and_relative_errors():
 
 @pytest.mark.gpu
 def test_search_on_gpu_meets_budget_and_is_minimal():
+    """The search through sta_forward on a 1024-token latent, against the
+    fp64 oracle: the reference is the oracle's whole-grid output (full
+    attention, itself checked against the library's dense attention), and the
+    chosen per-head windows, run together in one plan, match the oracle's
+    output for those windows element by element."""
+    import numpy as np
+
+    import oracle
     wl = Workload("ws", 1, 3, 64, 4, 16, 16, (2, 4, 4), ((1, 1, 1),) * 3, field_amplitude=1.0)
     q, k, v = make_inputs(wl, seed=5)
     # sharper scores in later heads: their attention is more local
     q = (q.float() * torch.tensor([0.5, 2.0, 6.0]).view(1, 3, 1, 1)).to(torch.bfloat16)
+    full = wl.with_(windows=(wl.grid,) * wl.Hh)
+    geom = lambda w: oracle.Geometry(w.B, w.Hh, w.d, w.T, w.H, w.W, tuple(w.tile), tuple(w.windows))
+    ref64, _ = oracle.forward(geom(full), q, k, v)
+    ref = torch.from_numpy(ref64).view(q.shape).cuda()
     q, k, v = (x.cuda() for x in (q, k, v))
+    sdpa = torch.nn.functional.scaled_dot_product_attention(q, k, v).double()
+    assert (sdpa - ref).abs().max().item() <= 2e-2 and (sdpa - ref).abs().mean().item() <= 2e-3
     cands = [(1, 1, 1), (1, 3, 3), (2, 3, 3), (2, 4, 4)]
     budget = 0.05
-    res = search_windows(q, k, v, wl.T, wl.H, wl.W, wl.tile, cands, budget)
-    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    res = search_windows(q, k, v, wl.T, wl.H, wl.W, wl.tile, cands, budget, reference=ref)
+    assert len(set(res.windows)) > 1  # the heads do not all take the same window
     # the chosen per-head windows, run together in one plan, stay within budget
     plan = sta.sta_plan_create(sta.Problem(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, wl.tile, res.windows))
-    o, _ = sta.sta_forward(plan, q, k, v, check=True)
+    o, lse = sta.sta_forward(plan, q, k, v, check=True)
     errs = relative_errors(o, ref)
     assert all(e <= budget for e in errs), errs
     # a head's output does not depend on the other heads' windows
     assert errs == pytest.approx(res.errors, rel=0, abs=1e-12)
+    # ... and it is the oracle's output for those windows, element by element
+    o_or, lse_or = oracle.forward(geom(wl.with_(windows=tuple(res.windows))), q, k, v)
+    e = np.abs(o.reshape(-1, wl.d).double().cpu().numpy() - o_or)
+    assert e.max() <= 2e-2 and e.mean() <= 2e-3, (e.max(), e.mean())
+    assert np.abs(lse.reshape(-1).double().cpu().numpy() - lse_or).max() <= 2e-3
     # and every cheaper candidate that was tried misses the budget for that head
     for h, w in enumerate(res.windows):
         for cand, e in res.tried:
