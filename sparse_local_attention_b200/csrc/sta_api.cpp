@@ -66,6 +66,8 @@ inline int window_start(int q, int w, int G) {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
 size_t tensor_bytes(const sta_plan_s *pl) {
   return (size_t)pl->g.B * pl->g.Hh * pl->g.N * pl->g.d * 2;
 }
@@ -79,17 +81,17 @@ size_t fwd_workspace(const sta_plan_s *pl) {
 }
 
 // Backward workspace: status word, then LSE*log2(e) and D = rowsum(dO*O), one
-// 128-float run per (batch, head, tile, query block), then (only when tiles
-// are not readable as boxes of the raster tensors) tile-major copies of Q, K, V
-// and dO.
-size_t bwd_vec_bytes(const sta_plan_s *pl) {
-  return (size_t)pl->g.B * pl->g.Hh * pl->g.n_tiles * pl->nqb * 128 * 4;
-}
+// 128-float run per (batch, head, tile, query block), then the two 4 KB
+// operand panels per query block that fold LSE and D into the dK/dV kernel's
+// S^T and dP^T products, then (only when tiles are not readable as boxes of
+// the raster tensors) tile-major copies of Q, K, V and dO.
+size_t bwd_blocks(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * pl->g.n_tiles * pl->nqb; }
+size_t bwd_vec_bytes(const sta_plan_s *pl) { return bwd_blocks(pl) * 128 * 4; }
+constexpr size_t kAugBytesPerBlock = 8192;
 // sta_forward_host workspace: device copies of Q, K, V, O and LSE (each at a
 // 256-byte boundary), then sta_forward's own workspace (status word first).
 constexpr int kHostGroups = 8;  // slice groups pipelined by sta_forward_host
 
-size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
 
 size_t lse_bytes(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * pl->g.N * 4; }
 
@@ -97,9 +99,11 @@ size_t host_copies_bytes(const sta_plan_s *pl) { return 4 * round256(tensor_byte
 
 size_t host_workspace(const sta_plan_s *pl) { return host_copies_bytes(pl) + fwd_workspace(pl); }
 
+size_t bwd_aug_offset(const sta_plan_s *pl) { return round256(kStatusBytes + 2 * bwd_vec_bytes(pl)); }
+size_t bwd_gather_offset(const sta_plan_s *pl) { return bwd_aug_offset(pl) + bwd_blocks(pl) * kAugBytesPerBlock; }
+
 size_t bwd_workspace(const sta_plan_s *pl) {
-  size_t b = kStatusBytes + 2 * bwd_vec_bytes(pl);
-  b = (b + 255) & ~size_t(255);
+  size_t b = bwd_gather_offset(pl);
   if (!pl->tiled && pl->kv_mode == sta::kKvTiled) b += 4 * tensor_bytes(pl);
   return b;
 }
@@ -825,7 +829,7 @@ sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void 
   const void *base[4] = {q, k, v, dout};
   const bool raster = pl->kv_mode == sta::kKvRaster;
   if (!pl->tiled && !raster) {
-    char *dst = ws + ((kStatusBytes + 2 * bwd_vec_bytes(pl) + 255) & ~size_t(255));
+    char *dst = ws + bwd_gather_offset(pl);
     for (int i = 0; i < 4; ++i) {
       sta::PermuteParams pp{};
       pp.g = pl->g;
@@ -852,6 +856,7 @@ sta_status sta_backward(sta_plan_t pl, const void *q, const void *k, const void 
   bp.oob_coord = raster ? pl->g.T * pl->g.B * pl->g.Hh : pl->g.B * pl->g.Hh * pl->g.N;
   bp.o = o, bp.dout = dout, bp.lse = lse;
   bp.lse2_t = lse2_t, bp.dd_t = dd_t;
+  bp.aug = reinterpret_cast<uint8_t *>(ws + bwd_aug_offset(pl));
   bp.dq = dq, bp.dk = dk, bp.dv = dv;
   bp.kv_list = pl->d_kv_list, bp.kv_count = pl->d_count, bp.kv_stride = pl->kv_stride;
   bp.inv_off = pl->d_inv_off, bp.inv_idx = pl->d_inv_idx;

@@ -55,6 +55,22 @@ struct Roles {
   static_assert(kCols % 32 == 0, "whole 32-column TMEM loads");
 };
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kAugPanelBytes = 4096, kAugBlockBytes = 2 * kAugPanelBytes;  // see BwdParams::aug
+// pairs of exponentials (of every 8) that the elementwise passes compute on
+// the FMA pipe (exp2_fma2) instead of the MUFU
+constexpr int kEmuBwd = 2;
+
+// x as two bf16 (hi, lo) with hi + lo = x to within 2^-16 relative: hi in
+// bits 0..15 (element 0 of the panel row), lo in bits 16..31 (element 1).
+__device__ __forceinline__ uint32_t hi_lo_bf16(float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+  return uint32_t(__bfloat16_as_ushort(hi)) | (uint32_t(__bfloat16_as_ushort(lo)) << 16);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -111,11 +127,18 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     const long long bt = run / p.nqb;  // bh * n_tiles + tile
     const int o = (int)(run - bt * p.nqb) * kBM + (int)(r - run * kBM);
     const int bh = (int)(bt / g.n_tiles), tile = (int)(bt - (long long)bh * g.n_tiles);
+    // row i of the block's two operand panels: lanes 0 / 1 write the two
+    // halves of the LSE panel's row, lanes 2 / 3 those of the D panel's row
+    const int i = (int)(r - run * kBM);
+    uint4 *cell = reinterpret_cast<uint4 *>(p.aug + run * kAugBlockBytes + (lane >> 1) * kAugPanelBytes +
+                                            (i / 8) * 256 + (lane & 1) * 128 + (i % 8) * 16);
     if (o >= g.tau) {
+      // rows past the tile's end: P = dS = 0 (LSE = +inf, D = 0)
       if (lane == 0) {
         p.dd_t[r] = 0.f;
         p.lse2_t[r] = INFINITY;
       }
+      if (lane < 4) *cell = make_uint4(lane == 0 ? hi_lo_bf16(-1e30f) : 0u, 0u, 0u, 0u);
       continue;
     }
     const long long tok = token_row(g, p.tiled, bh, tile, o);
@@ -131,10 +154,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    const float lse = p.lse[tok];
     if (lane == 0) {
       p.dd_t[r] = acc;
-      p.lse2_t[r] = p.lse[tok] * kLog2e;
+      p.lse2_t[r] = lse * kLog2e;
     }
+    // S^T + (-LSE / scale) times scale_log2 is S^T scale_log2 - LSE log2 e
+    if (lane < 4) *cell = make_uint4((lane & 1) ? 0u : hi_lo_bf16(lane == 0 ? -lse / p.scale : -acc), 0u, 0u, 0u);
   }
 }
 
@@ -153,10 +179,11 @@ struct DkvCfg {
   static constexpr bool kSep = D == 64;                    // P^T, dS^T in columns of their own
   using R = Roles<kSep ? 4 : 2>;                           // the in-place path assumes two warpgroups
   static constexpr int kStages = D == 128 ? 2 : 4;
-  static constexpr uint32_t kStage = 2 * kTile + 1024;     // Q, dO, LSE2[128], D[128]
+  static constexpr uint32_t kStage = 2 * kTile + kAugBlockBytes;  // Q, dO, the block's LSE and D panels
+  static constexpr uint32_t kOnes = kAugPanelBytes;               // panel of rows (1, 1, 0, ..., 0)
   // barriers: st_full[S] st_empty[S] kv_full kv_free s_full s_read p_ready pd_free acc_done acc_free drain
   static constexpr int kNumBars = 2 * kStages + 9;
-  static constexpr uint32_t kSmem = 2 * kTile + kStages * kStage + kNumBars * 8 + 64 + 1024;
+  static constexpr uint32_t kSmem = 2 * kTile + kStages * kStage + kOnes + kNumBars * 8 + 64 + 1024;
   static constexpr uint32_t kTmS = 0, kTmDP = 128;
   static constexpr uint32_t kTmP = kSep ? 256 : kTmS, kTmDS = kSep ? 320 : kTmDP;
   static constexpr uint32_t kTmDV = kSep ? 384 : 256, kTmDK = kTmDV + D;
@@ -175,8 +202,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *k_s = smem, *v_s = smem + C::kTile;
-  uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, lse2[128], dd[128]}
-  uint64_t *bars = reinterpret_cast<uint64_t *>(stages + C::kStages * C::kStage);
+  uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, LSE panel, D panel}
+  uint8_t *ones_s = stages + C::kStages * C::kStage;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ones_s + C::kOnes);
   uint64_t *st_full = bars, *st_empty = bars + C::kStages;
   uint64_t *kv_full = bars + 2 * C::kStages, *kv_free = kv_full + 1;
   uint64_t *s_full = kv_full + 2;    // S^T, dP^T of a chunk are in TMEM
@@ -210,6 +238,13 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  // the panel of ones: row k = (1, 1, 0, ..., 0) in the first half, zeros in
+  // the second (layout of BwdParams::aug)
+  for (int c = threadIdx.x; c < (int)(C::kOnes / 16); c += blockDim.x) {
+    const bool first_half = ((c * 16) % 256) < 128;
+    reinterpret_cast<uint4 *>(ones_s)[c] = make_uint4(first_half ? 0x3F803F80u : 0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -256,9 +291,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
             load_box<D>(p, &tmap_q, sb + pc * p.piece_rows * 128, c, &st_full[st]);
             load_box<D>(p, &tmap_do, sb + C::kTile + pc * p.piece_rows * 128, c, &st_full[st]);
           }
-          const long long lo = vec_run(p, bh, qt, qb);
-          bulk_load(sb + 2 * C::kTile, p.lse2_t + lo, 512, &st_full[st]);
-          bulk_load(sb + 2 * C::kTile + 512, p.dd_t + lo, 512, &st_full[st]);
+          const long long run = vec_run(p, bh, qt, qb) / kBM;
+          bulk_load(sb + 2 * C::kTile, p.aug + run * kAugBlockBytes, kAugBlockBytes, &st_full[st]);
           ++ld;
         }
         ++item_ctr;
@@ -276,6 +310,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       const uint64_t kd = smem_desc_sw128(smem_u32(k_s), 16, 1024), vd = smem_desc_sw128(smem_u32(v_s), 16, 1024);
       const uint64_t sk0 = smem_desc_sw128(smem_u32(stages), 16, 1024);              // K-major Q / dO
       const uint64_t sm0 = smem_desc_sw128(smem_u32(stages), C::kPanel, 1024);       // MN-major Q / dO
+      const uint64_t ones_d = smem_desc_plain(smem_u32(ones_s), 128, 256);
+      const uint64_t aug0 = smem_desc_plain(smem_u32(stages + 2 * C::kTile), 128, 256);  // stage 0's LSE panel
       uint32_t ld = 0, item_ctr = 0, p_waits = 0, r_waits = 0;
       bool ok = true, issued = false;
       // S^T = K Q^T and dP^T = V dO^T for the chunk in stage `st`
@@ -286,11 +322,15 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
           mma_ss(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
+        // + (-LSE / scale) per query column
+        mma_ss(tmem + C::kTmS, ones_d, aug0 + ((st * C::kStage) >> 4), idesc_ss, 1u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
           mma_ss(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
+        // - D per query column
+        mma_ss(tmem + C::kTmDP, ones_d, aug0 + ((st * C::kStage + kAugPanelBytes) >> 4), idesc_ss, 1u);
         mma_commit(s_full);
       };
       auto wait_stage = [&](uint32_t l) -> bool {
@@ -358,8 +398,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
     const int e = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const float sl2 = p.scale_log2;
-    uint32_t ld = 0, s_waits = 0, f_waits = 0, item_ctr = 0, gchunk = 0;
+    const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
+    uint32_t s_waits = 0, f_waits = 0, item_ctr = 0, gchunk = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
       int bh, ktile, kb, off0, nq;
@@ -367,32 +407,24 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       const int krow = kb * kBM + row;
       const bool row_valid = krow < g.tau;
       for (int i = 0; i < nq; ++i, ++gchunk) {
-        const uint32_t st = ld % C::kStages, ph = (ld / C::kStages) & 1;
-        bool okw = mbar_wait(&st_full[st], ph, ctl, kErrBwdWait) && mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
+        bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
-        // P^T and dS^T for this warpgroup's kCW query columns, packed to bf16
-        // (query rows past the tile's end have LSE = +inf: P = dS = 0 there).
-        const float4 *lse4 = reinterpret_cast<const float4 *>(stages + st * C::kStage + 2 * C::kTile) + (kCW / 4) * e;
-        const float4 *dd4 = lse4 + 32;
+        // P^T = 2^(S^T scale_log2) and dS^T = P^T dP^T for this warpgroup's
+        // kCW query columns, packed to bf16.  The MMAs have already added
+        // -LSE / scale to S^T and -D to dP^T from the operand panels (query
+        // rows past a tile's end get -1e30 and 0: P = dS = 0 there).
         uint32_t pp[kCW / 32][16], pd[kCW / 32][16];
-        // columns q0 .. q0 + 4 n - 1 of P^T / dS^T from raw S^T / dP^T bits
+        // columns q0 .. q0 + 2 n - 1 (of the warpgroup's kCW) from raw S^T / dP^T bits
         auto pds = [&](int q0, int n, const uint32_t *rs, const uint32_t *rd) {
 #pragma unroll
-          for (int v4 = 0; v4 < n; ++v4) {
-            const float4 l = lse4[q0 / 4 + v4], dv = dd4[q0 / 4 + v4];
-            const float ls[4] = {l.x, l.y, l.z, l.w}, ds[4] = {dv.x, dv.y, dv.z, dv.w};
-            float pr[4], dr[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              pr[h] = ex2_approx(fmaf(__uint_as_float(rs[4 * v4 + h]), sl2, -ls[h]));
-              dr[h] = pr[h] * (__uint_as_float(rd[4 * v4 + h]) - ds[h]);
-            }
-            const int w = (q0 + 4 * v4) / 2;  // packed column of the warpgroup's 32
-            pp[w >> 4][w & 15] = pack_bf16(pr[0], pr[1]);
-            pp[w >> 4][(w & 15) + 1] = pack_bf16(pr[2], pr[3]);
-            pd[w >> 4][w & 15] = pack_bf16(dr[0], dr[1]);
-            pd[w >> 4][(w & 15) + 1] = pack_bf16(dr[2], dr[3]);
+          for (int k = 0; k < n; ++k) {
+            const int w = q0 / 2 + k;  // packed column
+            const float2 t = mul2(make_float2(__uint_as_float(rs[2 * k]), __uint_as_float(rs[2 * k + 1])), sl2x2);
+            const float2 pr = (w % 8 >= 8 - kEmuBwd) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            const float2 dr = mul2(pr, make_float2(__uint_as_float(rd[2 * k]), __uint_as_float(rd[2 * k + 1])));
+            pp[w >> 4][w & 15] = pack_bf16(pr.x, pr.y);
+            pd[w >> 4][w & 15] = pack_bf16(dr.x, dr.y);
           }
         };
         if constexpr (C::kSep) {
@@ -412,7 +444,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
                 tc_fence_before();
                 warp_arrive(s_read, lane);
               }
-              pds(16 * h, 4, rs, rd);
+              pds(16 * h, 8, rs, rd);
             }
           }
         } else {
@@ -424,7 +456,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
             const uint32_t base = tmem + lane_off + 64 * e;
             quarters_pipelined(
                 base + C::kTmS, base + C::kTmDP,
-                [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) { pds(16 * qt, 4, rs, rd); },
+                [&](int qt, const uint32_t(&rs)[16], const uint32_t(&rd)[16]) { pds(16 * qt, 8, rs, rd); },
                 [&]() {});
           }
           // both warpgroups have read their S^T / dP^T columns before either
@@ -449,7 +481,6 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(p_ready, lane);
-        ++ld;
       }
       if (!ok) break;
       // epilogue: the first half of the warpgroups writes dV, the second half
@@ -716,7 +747,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
     const int e = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const float sl2 = p.scale_log2;
+    const float2 sl2x2 = make_float2(p.scale_log2, p.scale_log2);
     uint32_t s_waits = 0, f_waits = 0, item_ctr = 0, gchunk = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
@@ -725,6 +756,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
       const bool row_valid = qrow < g.tau;
       const long long lo = vec_run(p, it.bh, it.tile, it.qb) + row;
       const float lse2 = p.lse2_t[lo], dd = p.dd_t[lo];
+      const float2 nlse2 = make_float2(-lse2, -lse2), ndd = make_float2(-dd, -dd);
       for (int j = 0; j < it.nc; ++j, ++gchunk) {
         bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
@@ -750,19 +782,23 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
         uint32_t pd[kCW / 32][16];
 #pragma unroll
         for (int hf = 0; hf < kCW / 32; ++hf) {
-          float dr[32];
+          float2 dr[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float pv = ex2_approx(fmaf(__uint_as_float(rs[hf][c]), sl2, -lse2));
-            dr[c] = pv * (__uint_as_float(rd[hf][c]) - dd);
+          for (int k = 0; k < 16; ++k) {
+            const float2 t = fma2(make_float2(__uint_as_float(rs[hf][2 * k]), __uint_as_float(rs[hf][2 * k + 1])), sl2x2,
+                                  nlse2);
+            const float2 pr = (k % 8 >= 8 - kEmuBwd) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            dr[k] = mul2(pr, add2(make_float2(__uint_as_float(rd[hf][2 * k]), __uint_as_float(rd[hf][2 * k + 1])), ndd));
           }
           if (!whole) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (32 * hf + c >= kvalid) dr[c] = 0.f;
+            for (int k = 0; k < 16; ++k) {
+              if (32 * hf + 2 * k >= kvalid) dr[k].x = 0.f;
+              if (32 * hf + 2 * k + 1 >= kvalid) dr[k].y = 0.f;
+            }
           }
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) pd[hf][c / 2] = pack_bf16(dr[c], dr[c + 1]);
+          for (int k = 0; k < 16; ++k) pd[hf][k] = pack_bf16(dr[k].x, dr[k].y);
         }
         if (gchunk > 0) {
           // the dQ MMAs of the previous chunk have read dS

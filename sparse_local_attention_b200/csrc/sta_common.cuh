@@ -19,6 +19,35 @@ __device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
   return true;
 }
 
+// 2^x for two values at once on the FMA pipe, instead of the MUFU unit.
+// Cody and Waite's argument reduction: x = n + r with n = round(x) (adding
+// 1.5 * 2^23 rounds to an integer, which lands in the low mantissa bits) and r
+// in [-1/2, 1/2]; 2^r by a degree-3 polynomial in Horner form; n added to the
+// exponent field of the result.  The coefficients are this library's own
+// minimax fit of 2^r on [-1/2, 1/2] in relative error (fit_exp2_poly.py in
+// this directory): relative error <= 7.5e-5 for x >= -125 and <= 1.5e-4 down
+// to -126, far below the bf16 rounding of P that follows.  Inputs below -126
+// are clamped to -126 (2^-126 instead of a smaller value or 0): the softmax
+// adds these terms to a row sum >= 1 and multiplies them into V rows that are
+// zero for keys past the end of a list.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);
+  const float2 t = add2(x, magic);
+  const float2 r = sub2(x, sub2(t, magic));
+  float2 p = fma2(make_float2(kExp2C3, kExp2C3), r, make_float2(kExp2C2, kExp2C2));
+  p = fma2(p, r, make_float2(kExp2C1, kExp2C1));
+  p = fma2(p, r, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Token index (in the tensor's own order) of row `o` of tile `tile`.
 __device__ __forceinline__ long long token_row(const Geometry &g, int tiled, int bh, int tile, int o) {
   if (tiled) return (long long)bh * g.N + (long long)tile * g.tau + o;

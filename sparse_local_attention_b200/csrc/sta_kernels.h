@@ -72,7 +72,14 @@ struct BwdParams {
   int kv_mode, piece_rows, box_w, box_h, box_t, box_panels, oob_coord;
   const void *o, *dout;  // preprocess inputs
   const float *lse;      // forward LSE (natural log)
-  float *lse2_t, *dd_t;  // tile-major, pitch N + 128 per slice: LSE*log2(e), D = rowsum(dO*O)
+  float *lse2_t, *dd_t;  // one 128-float run per query block: LSE*log2(e), D = rowsum(dO*O)
+  // Per query block, two 4 KB K-major operand panels (no swizzle; 16 groups
+  // of 8 rows at 256 bytes, the two 8-element halves of a row 128 bytes
+  // apart): row q holds (hi, lo, 0, ..., 0) with hi + lo = -LSE_q*log2(e) /
+  // scale_log2 (first panel) and -D_q (second), hi and lo bf16.  The dK/dV
+  // kernel adds them to S^T and dP^T with one more K step against a panel of
+  // ones, so that its elementwise pass needs no per-query operand.
+  uint8_t *aug;
   void *dq, *dk, *dv;    // bf16 outputs
   const int32_t *kv_list, *kv_count;  // forward lists (dQ kernel)
   int kv_stride;

@@ -58,7 +58,7 @@ def test_kernel_register_budgets(tmp_path):
     res = _resources(tmp_path)
     for k in KERNELS:
         assert k in res, f"{k}: no ptxas report"
-    for k in ("sta_fwd_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel"):
+    for k in ("sta_fwd_kernel", "permute_kernel", "bwd_pre_kernel", "bwd_dq_kernel", "bwd_dkdv_kernel"):
         for mangled, regs, spill in res[k]:
             assert spill == 0, f"{k} ({mangled}) spills {spill} bytes"
     for mangled, regs, spill in res["sta_fwd_kernel"]:
@@ -67,5 +67,5 @@ def test_kernel_register_budgets(tmp_path):
         # head dim 64 runs 576 threads (96 registers), head dim 128 320 (168)
         cap = 96 if "ILi64E" in mangled else 168
         assert regs <= cap, (mangled, regs)
-        # spill store + load bytes: 28 (head dim 64) and 120 (head dim 128) today
-        assert spill <= 128, (mangled, spill)
+
+

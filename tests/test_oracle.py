@@ -28,8 +28,6 @@ import torch.nn.functional as F
 import oracle
 from oracle import Geometry
 
-torch.set_num_threads(4)
-
 
 def geom(T, H, W, tile, windows, B=1, d=16):
     return Geometry(B=B, Hh=len(windows), d=d, T=T, H=H, W=W, tile=tuple(tile),

@@ -5,7 +5,7 @@ import torch
 
 from sparse_local_attention_b200 import sta
 from sparse_local_attention_b200.window_search import clamped_keys, relative_errors, search_windows
-from sparse_local_attention_b200.workloads import Workload, make_inputs
+from sparse_local_attention_b200.workloads import Workload, positional_field
 
 
 def test_selection_rule_with_fake_forward():
@@ -68,10 +68,18 @@ def test_search_on_gpu_meets_budget_and_is_minimal():
     import numpy as np
 
     import oracle
+    # Attention that is local to a different extent in each head: queries and
+    # keys share the smooth positional field F (so q.k peaks where the two
+    # tokens are close), the query scaled by 0.5, 2 and 8 in the three heads,
+    # plus a little noise; values are N(0, 1).  (Seed 5, drawn in the order
+    # q noise, k noise, v.)
     wl = Workload("ws", 1, 3, 64, 4, 16, 16, (2, 4, 4), ((1, 1, 1),) * 3, field_amplitude=1.0)
-    q, k, v = make_inputs(wl, seed=5)
-    # sharper scores in later heads: their attention is more local
-    q = (q.float() * torch.tensor([0.5, 2.0, 6.0]).view(1, 3, 1, 1)).to(torch.bfloat16)
+    F = positional_field(wl)
+    gen = torch.Generator().manual_seed(5)
+    alphas = (0.5, 2.0, 8.0)
+    q = torch.stack([a * F + 0.1 * torch.randn(F.shape, generator=gen) for a in alphas])[None].to(torch.bfloat16)
+    k = torch.stack([F + 0.1 * torch.randn(F.shape, generator=gen) for _ in alphas])[None].to(torch.bfloat16)
+    v = torch.randn(1, 3, wl.N, wl.d, generator=gen).to(torch.bfloat16)
     full = wl.with_(windows=(wl.grid,) * wl.Hh)
     geom = lambda w: oracle.Geometry(w.B, w.Hh, w.d, w.T, w.H, w.W, tuple(w.tile), tuple(w.windows))
     ref64, _ = oracle.forward(geom(full), q, k, v)
@@ -80,9 +88,12 @@ def test_search_on_gpu_meets_budget_and_is_minimal():
     sdpa = torch.nn.functional.scaled_dot_product_attention(q, k, v).double()
     assert (sdpa - ref).abs().max().item() <= 2e-2 and (sdpa - ref).abs().mean().item() <= 2e-3
     cands = [(1, 1, 1), (1, 3, 3), (2, 3, 3), (2, 4, 4)]
-    budget = 0.05
+    # with these inputs the oracle's relative errors put the three heads'
+    # cheapest windows at 2x4x4 (the whole grid), 2x3x3 and 1x1x1, each
+    # candidate at least 0.04 away from the budget
+    budget = 0.28
     res = search_windows(q, k, v, wl.T, wl.H, wl.W, wl.tile, cands, budget, reference=ref)
-    assert len(set(res.windows)) > 1  # the heads do not all take the same window
+    assert len(set(res.windows)) == 3, res.windows  # the heads take different windows
     # the chosen per-head windows, run together in one plan, stay within budget
     plan = sta.sta_plan_create(sta.Problem(wl.B, wl.Hh, wl.d, wl.T, wl.H, wl.W, wl.tile, res.windows))
     o, lse = sta.sta_forward(plan, q, k, v, check=True)
