@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    // the whole warp issues (converged, warp-uniform operands; one elected lane per MMA)
+    {
       constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kBM, D, false, true);
       const uint64_t kd = smem_desc_sw128(smem_u32(k_s), 16, 1024), vd = smem_desc_sw128(smem_u32(v_s), 16, 1024);
@@ -320,28 +321,28 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kTmS, kd + off, sk0 + so + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
         // + (-LSE / scale) per query column
-        mma_ss(tmem + C::kTmS, ones_d, aug0 + ((st * C::kStage) >> 4), idesc_ss, 1u);
+        mma_ss_w(tmem + C::kTmS, ones_d, aug0 + ((st * C::kStage) >> 4), idesc_ss, 1u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
         // - D per query column
-        mma_ss(tmem + C::kTmDP, ones_d, aug0 + ((st * C::kStage + kAugPanelBytes) >> 4), idesc_ss, 1u);
-        mma_commit(s_full);
+        mma_ss_w(tmem + C::kTmDP, ones_d, aug0 + ((st * C::kStage + kAugPanelBytes) >> 4), idesc_ss, 1u);
+        mma_commit_w(s_full);
       };
       auto wait_stage = [&](uint32_t l) -> bool {
-        if (!mbar_wait(&st_full[l % C::kStages], (l / C::kStages) & 1, ctl, kErrBwdWait)) return false;
+        if (!mbar_wait_w(&st_full[l % C::kStages], (l / C::kStages) & 1, ctl, kErrBwdWait)) return false;
         tc_fence_after();
         return true;
       };
       for (int item = blockIdx.x; item < p.n_work_kv && ok; item += gridDim.x) {
         int bh, ktile, kb, off0, nq;
         item_info(item, bh, ktile, kb, off0, nq);
-        if (!mbar_wait(kv_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
+        if (!mbar_wait_w(kv_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
         tc_fence_after();
         if (!wait_stage(ld)) { ok = false; break; }
         issue_s(ld % C::kStages);
@@ -350,31 +351,31 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
           const uint32_t cur = ld + i, st = cur % C::kStages;
           if (C::kSep && i + 1 < nq) {
             // the next chunk's S^T / dP^T as soon as this chunk's have been read
-            if (!mbar_wait(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+            if (!mbar_wait_w(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
             ++r_waits;
             tc_fence_after();
             if (!wait_stage(cur + 1)) { ok = false; break; }
             issue_s((cur + 1) % C::kStages);
           }
-          if (!mbar_wait(p_ready, p_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          if (!mbar_wait_w(p_ready, p_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
           ++p_waits;
-          if (i == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          if (i == 0 && item_ctr > 0 && !mbar_wait_w(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
           tc_fence_after();
           // dV += P^T dO and dK += dS^T Q (queries are the contraction, 8 steps of 16)
           const uint32_t so = (st * C::kStage) >> 4, dso = (st * C::kStage + C::kTile) >> 4;
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             const uint32_t off = (kk * 16 * 128) >> 4;
-            mma_ts(tmem + C::kTmDV, tmem + C::kTmP + kk * 8, sm0 + dso + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_w(tmem + C::kTmDV, tmem + C::kTmP + kk * 8, sm0 + dso + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
             const uint32_t off = (kk * 16 * 128) >> 4;
-            mma_ts(tmem + C::kTmDK, tmem + C::kTmDS + kk * 8, sm0 + so + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_w(tmem + C::kTmDK, tmem + C::kTmDS + kk * 8, sm0 + so + off, idesc_acc, (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&st_empty[st]);
-          if (C::kSep) mma_commit(pd_free);
-          if (i + 1 == nq) mma_commit(kv_free);
+          mma_commit_w(&st_empty[st]);
+          if (C::kSep) mma_commit_w(pd_free);
+          if (i + 1 == nq) mma_commit_w(kv_free);
           if (!C::kSep && i + 1 < nq) {
             // P^T / dS^T live in the S^T / dP^T columns: the next S^T / dP^T
             // are issued after the MMAs that read them (in-order execution)
@@ -384,11 +385,11 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
         }
         if (!ok) break;
         ld += nq;
-        mma_commit(acc_done);
+        mma_commit_w(acc_done);
         ++item_ctr;
       }
       if (!ok && issued) {
-        mma_commit(drain);
+        mma_commit_w(drain);
         drain_wait(drain, 0);
       }
     }
@@ -672,7 +673,8 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
       if (item_ctr > 0) drain_wait(q_full, (item_ctr - 1) & 1);
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    // the whole warp issues (converged, warp-uniform operands; one elected lane per MMA)
+    {
       constexpr uint32_t idesc_ss = idesc_bf16_f32(kBM, kBM, false, false);
       constexpr uint32_t idesc_dq = idesc_bf16_f32(kBM, D, false, true);
       const uint64_t qd = smem_desc_sw128(smem_u32(q_s), 16, 1024), dod = smem_desc_sw128(smem_u32(do_s), 16, 1024);
@@ -683,61 +685,61 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
       // S = Q K^T and dP = dO V^T for chunk j (ring loads lk = K_j, lk + 1 = V_j)
       auto issue_s = [&](uint32_t lk) -> bool {
         const uint32_t lv = lk + 1, ks = lk % C::kSlots, vs = lv % C::kSlots;
-        if (!mbar_wait(&full[ks], (lk / C::kSlots) & 1, ctl, kErrBwdWait) ||
-            !mbar_wait(&full[vs], (lv / C::kSlots) & 1, ctl, kErrBwdWait))
+        if (!mbar_wait_w(&full[ks], (lk / C::kSlots) & 1, ctl, kErrBwdWait) ||
+            !mbar_wait_w(&full[vs], (lv / C::kSlots) & 1, ctl, kErrBwdWait))
           return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::kTmS, qd + off, sk0 + ((ks * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kTmS, qd + off, sk0 + ((ks * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanel + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::kTmDP, dod + off, sk0 + ((vs * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
+          mma_ss_w(tmem + C::kTmDP, dod + off, sk0 + ((vs * C::kTile) >> 4) + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full);
-        mma_commit(&empty[vs]);  // V is read by dP only
+        mma_commit_w(s_full);
+        mma_commit_w(&empty[vs]);  // V is read by dP only
         return true;
       };
       for (int item = blockIdx.x; item < p.n_work_q && ok; item += gridDim.x) {
         const Item it = item_info(item);
-        if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
+        if (!mbar_wait_w(q_full, item_ctr & 1, ctl, kErrBwdWait)) { ok = false; break; }
         tc_fence_after();
         if (!issue_s(ld)) { ok = false; break; }
         issued = true;
-        if (it.nc == 1) mma_commit(q_free);
+        if (it.nc == 1) mma_commit_w(q_free);
         for (int j = 0; j < it.nc && ok; ++j) {
           const uint32_t lk = ld + 2 * j;
           if (j + 1 < it.nc) {
             // the next chunk's S / dP as soon as this chunk's have been read
-            if (!mbar_wait(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+            if (!mbar_wait_w(s_read, r_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
             ++r_waits;
             tc_fence_after();
             if (!issue_s(lk + 2)) { ok = false; break; }
-            if (j + 2 == it.nc) mma_commit(q_free);  // Q and dO are no longer read
+            if (j + 2 == it.nc) mma_commit_w(q_free);  // Q and dO are no longer read
           }
-          if (!mbar_wait(ds_ready, ds_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          if (!mbar_wait_w(ds_ready, ds_waits & 1, ctl, kErrBwdWait)) { ok = false; break; }
           ++ds_waits;
-          if (j == 0 && item_ctr > 0 && !mbar_wait(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
+          if (j == 0 && item_ctr > 0 && !mbar_wait_w(acc_free, (item_ctr - 1) & 1, ctl, kErrBwdWait)) { ok = false; break; }
           tc_fence_after();
           // dQ += dS K (keys are the contraction)
           const uint32_t ks = lk % C::kSlots;
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk)
-            mma_ts(tmem + C::kTmDQ, tmem + C::kTmDS + kk * 8, sm0 + ((ks * C::kTile + kk * 16 * 128) >> 4), idesc_dq,
+            mma_ts_w(tmem + C::kTmDQ, tmem + C::kTmDS + kk * 8, sm0 + ((ks * C::kTile + kk * 16 * 128) >> 4), idesc_dq,
                    (j > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[ks]);
-          mma_commit(ds_free);
+          mma_commit_w(&empty[ks]);
+          mma_commit_w(ds_free);
         }
         if (!ok) break;
         ld += 2 * it.nc;
-        mma_commit(acc_done);
+        mma_commit_w(acc_done);
         ++item_ctr;
       }
       if (!ok && issued) {
-        mma_commit(drain);
+        mma_commit_w(drain);
         drain_wait(drain, 0);
       }
     }

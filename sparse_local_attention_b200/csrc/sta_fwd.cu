@@ -258,7 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs this loop (converged, operands warp-uniform); one
+    // elected lane issues each MMA and commit.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
       const uint32_t slots_addr = smem_u32(slots), q_addr = smem_u32(q_smem);
@@ -279,9 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::kPanelBytes + (kk % 4) * 32) >> 4;
-          mma_ss(d_tm, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss_w(d_tm, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&s_full[x]);
+        mma_commit_w(&s_full[x]);
       };
       // O_X += P_X V for the V chunk in ring slot `slot`, in two halves of 64
       // keys: the first is issued as soon as the softmax has written P for
@@ -291,18 +293,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_tm = tmem + C::kTmO0 + x * D, p_tm = tmem + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < kBN / 32; ++kk)
-          mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
-        if (!mbar_wait(&p_ready[x], ph, ctl, kErrWaitMma)) return false;
+          mma_ts_w(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        if (!mbar_wait_w(&p_ready[x], ph, ctl, kErrWaitMma)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = kBN / 32; kk < kBN / 16; ++kk)
-          mma_ts(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, 1u);
-        mma_commit(&pv_done[x]);
+          mma_ts_w(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, 1u);
+        mma_commit_w(&pv_done[x]);
         return true;
       };
       auto wait_slot = [&](uint32_t slot_ld) -> bool {
         const uint32_t slot = slot_ld % C::kSlots, phase = (slot_ld / C::kSlots) & 1;
-        if (!mbar_wait(&full[slot], phase, ctl, kErrWaitMma)) return false;
+        if (!mbar_wait_w(&full[slot], phase, ctl, kErrWaitMma)) return false;
         tc_fence_after();
         return true;
       };
@@ -311,37 +313,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
           const ItemInfo it = decode_item<kMode>(p, item);
           const int nx = it.has_b ? 2 : 1;
-          if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
+          if (!mbar_wait_w(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
           tc_fence_after();
           // chunk 0: S_A(0) [, S_B(0)]
           const uint32_t k0 = ld;
           if (!wait_slot(k0)) { ok = false; break; }
           for (int x = 0; x < nx; ++x) mma_s(x, x, k0 % C::kSlots);
           issued = true;
-          mma_commit(&empty[k0 % C::kSlots]);
-          if (it.nc == 1) mma_commit(q_free);
+          mma_commit_w(&empty[k0 % C::kSlots]);
+          if (it.nc == 1) mma_commit_w(q_free);
           for (int j = 0; j < it.nc && ok; ++j) {
             const uint32_t vj = k0 + 2 * j + 1, kn = k0 + 2 * j + 2;  // V_j, K_{j+1} load indices
             for (int x = 0; x < nx; ++x) {
               const uint32_t ph = p_waits[x] & 1;
-              if (!mbar_wait(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
+              if (!mbar_wait_w(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
                 // the previous item of this block has read O_X in its epilogue
-                if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+                if (!mbar_wait_w(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
                 ++o_waits[x];
                 tc_fence_after();
               }
               if (x == 0 && !wait_slot(vj)) { ok = false; break; }
               if (!mma_pv(x, vj % C::kSlots, j == 0, ph)) { ok = false; break; }
-              if (x == nx - 1) mma_commit(&empty[vj % C::kSlots]);
+              if (x == nx - 1) mma_commit_w(&empty[vj % C::kSlots]);
               if (j + 1 < it.nc) {
                 if (x == 0 && !wait_slot(kn)) { ok = false; break; }
                 mma_s(x, x, kn % C::kSlots);
                 if (x == nx - 1) {
-                  mma_commit(&empty[kn % C::kSlots]);
-                  if (j + 2 == it.nc) mma_commit(q_free);
+                  mma_commit_w(&empty[kn % C::kSlots]);
+                  if (j + 2 == it.nc) mma_commit_w(q_free);
                 }
               }
             }
@@ -354,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int item = blockIdx.x; item < p.n_work && ok; item += gridDim.x) {
           const ItemInfo it = decode_item<kMode>(p, item);
           const int nx = it.split ? 2 : 1;
-          if (!mbar_wait(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
+          if (!mbar_wait_w(q_full, item_ctr & 1, ctl, kErrWaitMma)) { ok = false; break; }
           tc_fence_after();
           uint32_t l = ld, kslot = 0, vslot = 0;
           int s_left = it.nc;  // S groups still to issue (one per chunk)
@@ -364,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             slot = l++;
             return true;
           };
-          auto release = [&](uint32_t slot) { mma_commit(&empty[slot % C::kSlots]); };
+          auto release = [&](uint32_t slot) { mma_commit_w(&empty[slot % C::kSlots]); };
           auto s_group_done = [&]() {
-            if (--s_left == 0) mma_commit(q_free);  // Q is no longer read
+            if (--s_left == 0) mma_commit_w(q_free);  // Q is no longer read
           };
           // first chunk of each warpgroup
           for (int x = 0; x < nx && ok; ++x) {
@@ -380,12 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < nx; ++x) {
               if (j >= it.n(x)) continue;
               const uint32_t ph = p_waits[x] & 1;
-              if (!mbar_wait(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
+              if (!mbar_wait_w(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
                 // the previous item of this warpgroup has read O_X in its epilogue
-                if (!mbar_wait(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
+                if (!mbar_wait_w(&o_free[x], o_waits[x] & 1, ctl, kErrWaitMma)) { ok = false; break; }
                 ++o_waits[x];
                 tc_fence_after();
               }
@@ -406,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       if (!ok && issued) {
         // Wait for every MMA already issued before TMEM is released.
-        mma_commit(drain);
+        mma_commit_w(drain);
         drain_wait(drain, 0);
       }
     }
