@@ -509,7 +509,9 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
         for (int b = 0; b < g.B; ++b)
           for (int t = 0; t < g.n_tiles; ++t)
             for (int qb = 0; qb < nqb; ++qb) pl->work_q.push_back(make_int2(b * g.Hh + h, t * nqb + qb));
-      // dK/dV: one 128-row key block per item, longest inverse list first.
+      // dK/dV: one 128-row key block per item, slice by slice (the key blocks
+      // running at the same time then read the query tiles of one slice,
+      // which stay in L2), within a slice longest inverse list first.
       struct KvItem { int len, bh, key; };
       std::vector<KvItem> items;
       items.reserve((size_t)g.B * g.Hh * g.n_tiles * nqb);
@@ -519,7 +521,8 @@ sta_status sta_plan_create(const sta_problem *prob, sta_plan_t *out) {
             const int32_t *off = &pl->inv_off[(size_t)h * (g.n_tiles + 1) + t];
             for (int kb = 0; kb < nqb; ++kb) items.push_back({off[1] - off[0], b * g.Hh + h, t * nqb + kb});
           }
-      std::stable_sort(items.begin(), items.end(), [](const KvItem &a, const KvItem &c) { return a.len > c.len; });
+      std::stable_sort(items.begin(), items.end(),
+                       [](const KvItem &a, const KvItem &c) { return a.bh != c.bh ? a.bh < c.bh : a.len > c.len; });
       for (const KvItem &it : items) pl->work_kv.push_back(make_int2(it.bh, it.key));
     }
   } catch (const std::bad_alloc &) {

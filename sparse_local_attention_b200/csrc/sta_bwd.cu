@@ -56,9 +56,9 @@ struct Roles {
 };
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kAugPanelBytes = 4096, kAugBlockBytes = 2 * kAugPanelBytes;  // see BwdParams::aug
-// pairs of exponentials (of every 8) that the elementwise passes compute on
-// the FMA pipe (exp2_fma2) instead of the MUFU
-constexpr int kEmuBwd = 2;
+// pairs of exponentials (of every 8) that the dK/dV and the dQ elementwise
+// passes compute on the FMA pipe (exp2_fma2) instead of the MUFU
+constexpr int kEmuDkdv = 0, kEmuDq = 0;
 
 // x as two bf16 (hi, lo) with hi + lo = x to within 2^-16 relative: hi in
 // bits 0..15 (element 0 of the panel row), lo in bits 16..31 (element 1).
@@ -422,31 +422,31 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
           for (int k = 0; k < n; ++k) {
             const int w = q0 / 2 + k;  // packed column
             const float2 t = mul2(make_float2(__uint_as_float(rs[2 * k]), __uint_as_float(rs[2 * k + 1])), sl2x2);
-            const float2 pr = (w % 8 >= 8 - kEmuBwd) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            const float2 pr = (w % 8 >= 8 - kEmuDkdv) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
             const float2 dr = mul2(pr, make_float2(__uint_as_float(rd[2 * k]), __uint_as_float(rd[2 * k + 1])));
             pp[w >> 4][w & 15] = pack_bf16(pr.x, pr.y);
             pd[w >> 4][w & 15] = pack_bf16(dr.x, dr.y);
           }
         };
         if constexpr (C::kSep) {
-          // S^T and dP^T are read, then their columns released at once: the MMA
-          // warp computes the next chunk's while this one is done
-          // (16 columns of each at a time, so few registers stay live).
+          // S^T and dP^T are read in one batch and their columns released at
+          // once, before any arithmetic: the MMA warp computes the next
+          // chunk's S^T / dP^T while this one is worked on.
+          static_assert(kCW == 32, "one 32-column load of each");
           if (okw) {
             tc_fence_after();
             const uint32_t base = tmem + lane_off + kCW * e;
-#pragma unroll
-            for (int h = 0; h < kCW / 16; ++h) {
-              uint32_t rs[16], rd[16];
-              tmem_ld16(base + C::kTmS + 16 * h, rs);
-              tmem_ld16(base + C::kTmDP + 16 * h, rd);
-              tmem_ld_wait_regs(rs, rd);
-              if (h + 1 == kCW / 16 && i + 1 < nq) {
-                tc_fence_before();
-                warp_arrive(s_read, lane);
-              }
-              pds(16 * h, 8, rs, rd);
+            uint32_t rs[32], rd[32];
+            tmem_ld32(base + C::kTmS, rs);
+            tmem_ld32(base + C::kTmDP, rd);
+            tmem_ld_wait();
+            reg_fence32(rs);
+            reg_fence32(rd);
+            if (i + 1 < nq) {
+              tc_fence_before();
+              warp_arrive(s_read, lane);
             }
+            pds(0, 16, rs, rd);
           }
         } else {
           // P^T / dS^T are written over S^T / dP^T, so their columns are not
@@ -789,7 +789,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
           for (int k = 0; k < 16; ++k) {
             const float2 t = fma2(make_float2(__uint_as_float(rs[hf][2 * k]), __uint_as_float(rs[hf][2 * k + 1])), sl2x2,
                                   nlse2);
-            const float2 pr = (k % 8 >= 8 - kEmuBwd) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
+            const float2 pr = (k % 8 >= 8 - kEmuDq) ? exp2_fma2(t) : make_float2(ex2_approx(t.x), ex2_approx(t.y));
             dr[k] = mul2(pr, add2(make_float2(__uint_as_float(rd[hf][2 * k]), __uint_as_float(rd[hf][2 * k + 1])), ndd));
           }
           if (!whole) {

@@ -107,10 +107,10 @@ def test_backward_items(name):
     dq, _ = sta.sta_plan_work_items(plan, sta.STA_WORK_DQ)
     assert sorted(map(tuple, kv.tolist())) == every
     assert sorted(map(tuple, dq.tolist())) == every
-    # dK/dV items: longest inverse list first
+    # dK/dV items: slice by slice, within a slice longest inverse list first
     inv = [sta.sta_plan_q_tiles(plan, h)[0] for h in range(wl.Hh)]
-    lens = [int(inv[s % wl.Hh][blk // nb + 1] - inv[s % wl.Hh][blk // nb]) for s, blk in kv.tolist()]
-    assert lens == sorted(lens, reverse=True)
+    keyed = [(s, -int(inv[s % wl.Hh][blk // nb + 1] - inv[s % wl.Hh][blk // nb])) for s, blk in kv.tolist()]
+    assert keyed == sorted(keyed)
     # dQ items: costliest heads first
     count = [len(sta.sta_plan_kv_tiles(plan, h)[0]) for h in range(wl.Hh)]
     costs = [count[s % wl.Hh] for s, _ in dq.tolist()]

@@ -36,7 +36,8 @@ MUTANTS = [
     ("lone_blocks_first", "    pl->work.insert(pl->work.end(), lone_items.begin(), lone_items.end());",
      "    pl->work.insert(pl->work.begin(), lone_items.begin(), lone_items.end());"),
     ("forward_cost_ascending", "return cost(a) > cost(b);", "return cost(a) < cost(b);"),
-    ("dkdv_shortest_first", "return a.len > c.len;", "return a.len < c.len;"),
+    ("dkdv_shortest_first", "a.bh < c.bh : a.len > c.len;", "a.bh < c.bh : a.len < c.len;"),
+    ("dkdv_slices_interleaved", "return a.bh != c.bh ? a.bh < c.bh : a.len > c.len;", "return a.len > c.len;"),
     ("dq_last_block_missing", "            for (int qb = 0; qb < nqb; ++qb) pl->work_q.push_back(",
      "            for (int qb = 0; qb + 1 < nqb || (nqb == 1 && qb < 0); ++qb) pl->work_q.push_back("),
     ("host_groups_shifted", "pl->group_slice[gi] = (int)((long long)slices * gi / groups);",
