@@ -96,9 +96,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
 
 // mbar_wait for a whole warp: every lane waits, and the result is the same in
 // all of them (false if any lane's wait failed), so that the warp stays
-// converged for the warp-wide MMA issue below.
+// converged for the warp-wide MMA issue below.  Every branch depends on a warp
+// vote, so the compiler sees uniform control flow: a wait whose phase has
+// already completed costs one probe and one vote (the per-lane loop of
+// mbar_wait costs ~120 cycles on B200 even then).
 __device__ __forceinline__ bool mbar_wait_w(uint64_t *bar, uint32_t parity, const WaitCtl &ctl, int code) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl, code));
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+  const long long limit = (long long)(ctl.limit_ns * 2ull);
+  const long long t0 = clock64();
+  while (true) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if (__any_sync(0xffffffffu, *ctl.abort != 0)) return false;
+    if (__any_sync(0xffffffffu, clock64() - t0 >= limit)) {
+      if ((threadIdx.x & 31) == 0) {
+        *ctl.abort = 1;
+        atomicCAS(ctl.status, 0, code);
+      }
+      __syncwarp();
+      return false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- TMA
@@ -344,51 +361,12 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // Packed two-wide fp32 arithmetic (sm_100a): one instruction does the same
-// operation on both halves of a 64-bit register pair, each rounded to nearest.
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
-      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
-      "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
-      : "=l"(d)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 ra, rb;\n\t"
-      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
-      "add.rn.f32x2 %0, ra, rb;\n\t}"
-      : "=l"(d)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 ra, rb;\n\t"
-      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
-      "mul.rn.f32x2 %0, ra, rb;\n\t}"
-      : "=l"(d)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-  uint64_t d;
-  asm("{\n\t.reg .b64 ra, rb;\n\t"
-      "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
-      "sub.rn.f32x2 %0, ra, rb;\n\t}"
-      : "=l"(d)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
-  return r;
-}
+// operation on both halves of a register pair, each rounded to nearest.  The
+// compiler's own builtins, so that it allocates the pairs itself.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
 
 // Register budget of the calling warpgroup (all four warps must execute it):
 // give back registers down to N per thread, or take more up to N.

@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       const int krow = kb * kBM + row;
       const bool row_valid = krow < g.tau;
       for (int i = 0; i < nq; ++i, ++gchunk) {
-        bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
+        bool okw = mbar_wait_w(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
         // P^T = 2^(S^T scale_log2) and dS^T = P^T dP^T for this warpgroup's
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
         if (!okw) { ok = false; break; }
         if (C::kSep && gchunk > 0) {
           // the dV / dK MMAs of the previous chunk have read P^T / dS^T
-          bool okf = mbar_wait(pd_free, f_waits & 1, ctl, kErrBwdWait);
+          bool okf = mbar_wait_w(pd_free, f_waits & 1, ctl, kErrBwdWait);
           ++f_waits;
           okf = __all_sync(0xffffffffu, okf);
           if (!okf) { ok = false; break; }
@@ -486,7 +486,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       if (!ok) break;
       // epilogue: the first half of the warpgroups writes dV, the second half
       // scale * dK (rows of this key block), each warpgroup kOut columns
-      bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
+      bool oke = mbar_wait_w(acc_done, item_ctr & 1, ctl, kErrBwdWait);
       oke = __all_sync(0xffffffffu, oke);
       if (!C::kSep) oke = named_bar_and(1, 32 * kMathWarps, oke);
       if (!oke) { ok = false; break; }
@@ -760,7 +760,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
       const float lse2 = p.lse2_t[lo], dd = p.dd_t[lo];
       const float2 nlse2 = make_float2(-lse2, -lse2), ndd = make_float2(-dd, -dd);
       for (int j = 0; j < it.nc; ++j, ++gchunk) {
-        bool okw = mbar_wait(s_full, s_waits & 1, ctl, kErrBwdWait);
+        bool okw = mbar_wait_w(s_full, s_waits & 1, ctl, kErrBwdWait);
         ++s_waits;
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
@@ -804,7 +804,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
         }
         if (gchunk > 0) {
           // the dQ MMAs of the previous chunk have read dS
-          bool okf = mbar_wait(ds_free, f_waits & 1, ctl, kErrBwdWait);
+          bool okf = mbar_wait_w(ds_free, f_waits & 1, ctl, kErrBwdWait);
           ++f_waits;
           okf = __all_sync(0xffffffffu, okf);
           if (!okf) { ok = false; break; }
@@ -817,7 +817,7 @@ __global__ void __launch_bounds__(DqCfg<D>::R::kThreads, 1)
         warp_arrive(ds_ready, lane);
       }
       if (!ok) break;
-      bool oke = mbar_wait(acc_done, item_ctr & 1, ctl, kErrBwdWait);
+      bool oke = mbar_wait_w(acc_done, item_ctr & 1, ctl, kErrBwdWait);
       oke = __all_sync(0xffffffffu, oke);
       if (!oke) { ok = false; break; }
       tc_fence_after();

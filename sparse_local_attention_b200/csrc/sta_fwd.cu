@@ -436,11 +436,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < it.n(x) && ok; ++j) {
-        bool okw = mbar_wait(&s_full[x], s_waits & 1, ctl, kErrWaitSoftmax);
+        bool okw = mbar_wait_w(&s_full[x], s_waits & 1, ctl, kErrWaitSoftmax);
         ++s_waits;
         if (okw && j > 0) {
           // O_X holds every chunk before j once P V(j-1) is done
-          okw = mbar_wait(&pv_done[x], pv_waits & 1, ctl, kErrWaitSoftmax);
+          okw = mbar_wait_w(&pv_done[x], pv_waits & 1, ctl, kErrWaitSoftmax);
           ++pv_waits;
         }
         okw = __all_sync(0xffffffffu, okw);
@@ -529,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue: O_X / l -> bf16 row, LSE
       bool oke = false;
       if (ok) {
-        oke = mbar_wait(&pv_done[x], pv_waits & 1, ctl, kErrWaitEpilogue);
+        oke = mbar_wait_w(&pv_done[x], pv_waits & 1, ctl, kErrWaitEpilogue);
         ++pv_waits;
         oke = __all_sync(0xffffffffu, oke);
       }
