@@ -62,7 +62,13 @@ struct FwdCfg {
   static constexpr int kSlots = (D == 128 ? 4 : 8) + (2 - kNumQ);
   static constexpr uint32_t kTmO0 = 256;  // O_X at kTmO0 + X * D; S_X at 128 * X
   static constexpr uint32_t kTmCols = 512;
-  // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain p_half[2]
+  // P of a chunk's first kLeadKeys keys is published on its own (p_lead) and
+  // its share of P V issued at once, so that only the rest of P V stands
+  // between the end of the softmax and the next S (measured on B200: a lead of
+  // 96 keys is the faster at head dim 128, 64 keys at head dim 64).
+  static constexpr int kLeadKeys = D == 128 ? 96 : 64;
+  static_assert(kLeadKeys % 32 == 0 && kLeadKeys < kBN, "whole 32-key groups of P");
+  // barriers: full[S] empty[S] q_full q_free s_full[2] p_ready[2] pv_done[2] o_free[2] drain p_lead[2]
   static constexpr int kNumBars = 2 * kSlots + 13;
   static constexpr uint32_t kMiscBytes = 64 + 4 * 128 * 4;  // tmem address, abort flag, m/l exchange
   static constexpr uint32_t kListBytes = kMaxCoords * 16;
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *pv_done = p_ready + 2;          // [2]
   uint64_t *o_free = pv_done + 2;           // [2]
   uint64_t *drain = o_free + 2;
-  uint64_t *p_half = drain + 1;             // [2] P of the chunk's first 64 keys written
+  uint64_t *p_lead = drain + 1;             // [2] P of the chunk's first kLeadKeys keys written
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::kNumBars);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *ml_xchg = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(tmem_slot) + 64);  // [m0 m1 l0 l1][128]
@@ -146,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
       mbar_init(&p_ready[x], 4);  // the four warps of the block's warpgroup
-      mbar_init(&p_half[x], 4);
+      mbar_init(&p_lead[x], 4);
       mbar_init(&pv_done[x], 1);
       mbar_init(&o_free[x], 4);
     }
@@ -285,19 +291,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit_w(&s_full[x]);
       };
-      // O_X += P_X V for the V chunk in ring slot `slot`, in two halves of 64
-      // keys: the first is issued as soon as the softmax has written P for
-      // those keys, the second (and the pv_done commit) once all of P is there.
+      // O_X += P_X V for the V chunk in ring slot `slot`, in two parts: the
+      // first kLeadKeys keys as soon as the softmax has written P for them, the
+      // rest (and the pv_done commit) once all of P is there.
       auto mma_pv = [&](int x, uint32_t slot, bool first, uint32_t ph) -> bool {
         const uint64_t vd = vdesc0 + ((slot * C::kTileBytes) >> 4);
         const uint32_t o_tm = tmem + C::kTmO0 + x * D, p_tm = tmem + 128 * x;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 32; ++kk)
+        for (int kk = 0; kk < C::kLeadKeys / 16; ++kk)
           mma_ts_w(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
         if (!mbar_wait_w(&p_ready[x], ph, ctl, kErrWaitMma)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+        for (int kk = C::kLeadKeys / 16; kk < kBN / 16; ++kk)
           mma_ts_w(o_tm, p_tm + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv, 1u);
         mma_commit_w(&pv_done[x]);
         return true;
@@ -324,9 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it.nc == 1) mma_commit_w(q_free);
           for (int j = 0; j < it.nc && ok; ++j) {
             const uint32_t vj = k0 + 2 * j + 1, kn = k0 + 2 * j + 2;  // V_j, K_{j+1} load indices
+            // V_j and K_{j+1} land long before they are used: wait for them here,
+            // while the softmax works, not between P V(j) and S(j + 1)
+            if (!wait_slot(vj) || (j + 1 < it.nc && !wait_slot(kn))) { ok = false; break; }
             for (int x = 0; x < nx; ++x) {
               const uint32_t ph = p_waits[x] & 1;
-              if (!mbar_wait_w(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
+              if (!mbar_wait_w(&p_lead[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
@@ -335,11 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++o_waits[x];
                 tc_fence_after();
               }
-              if (x == 0 && !wait_slot(vj)) { ok = false; break; }
               if (!mma_pv(x, vj % C::kSlots, j == 0, ph)) { ok = false; break; }
               if (x == nx - 1) mma_commit_w(&empty[vj % C::kSlots]);
               if (j + 1 < it.nc) {
-                if (x == 0 && !wait_slot(kn)) { ok = false; break; }
                 mma_s(x, x, kn % C::kSlots);
                 if (x == nx - 1) {
                   mma_commit_w(&empty[kn % C::kSlots]);
@@ -382,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < nx; ++x) {
               if (j >= it.n(x)) continue;
               const uint32_t ph = p_waits[x] & 1;
-              if (!mbar_wait_w(&p_half[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
+              if (!mbar_wait_w(&p_lead[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
               tc_fence_after();
               if (j == 0 && x_items[x] > 0) {
@@ -485,9 +492,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = m_new;
 
         // P = exp2(S * scale_log2 - m) as bf16 over the consumed S columns, row
-        // sum.  The first 64 keys are published on their own (p_half) so that
-        // half of P V runs while the rest of P is formed; O is rescaled (rarely)
-        // before that, once the first half of S is no longer held.
+        // sum.  The first kLeadKeys keys are published on their own (p_lead) so
+        // that their share of P V runs while the rest of P is formed; O is
+        // rescaled (rarely) before that, once the first half of S is no longer
+        // held.
         float ls[8];
 #pragma unroll
         for (int a = 0; a < 8; ++a) ls[a] = 0.f;
@@ -502,22 +510,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[i / 2] = pack_bf16(p0, p1);
           }
           tmem_st16(tmem + lane_off + s_col + c * 16, pk);
-          if (c == 1) {
-            if (warp_resc) {
-              // O holds every chunk before j (P V(j-1) finished before S(j))
+          if (c == 1 && warp_resc) {
+            // O holds every chunk before j (P V(j-1) finished before S(j))
 #pragma unroll 1
-              for (int oc = 0; oc < D / 16; ++oc) {
-                uint32_t r[16];
-                tmem_ld16(tmem + lane_off + o_col + oc * 16, r);
-                tmem_ld_wait();
+            for (int oc = 0; oc < D / 16; ++oc) {
+              uint32_t r[16];
+              tmem_ld16(tmem + lane_off + o_col + oc * 16, r);
+              tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                tmem_st16(tmem + lane_off + o_col + oc * 16, r);
-              }
+              for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st16(tmem + lane_off + o_col + oc * 16, r);
             }
+          }
+          if (c == C::kLeadKeys / 32 - 1) {
             tmem_st_wait();
             tc_fence_before();
-            warp_arrive(&p_half[x], lane);
+            warp_arrive(&p_lead[x], lane);
           }
         }
         l = l * alpha + (((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7])));
