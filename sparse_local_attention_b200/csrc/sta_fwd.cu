@@ -388,6 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < it.n(0) && ok; ++j) {
             for (int x = 0; x < nx; ++x) {
               if (j >= it.n(x)) continue;
+              // V(j) and K(j + 1) of this stream, waited for while the softmax
+              // works rather than between P V(j) and S(j + 1)
+              if (!take(vslot) || (j + 1 < it.n(x) && !take(kslot))) { ok = false; break; }
               const uint32_t ph = p_waits[x] & 1;
               if (!mbar_wait_w(&p_lead[x], ph, ctl, kErrWaitMma)) { ok = false; break; }
               ++p_waits[x];
@@ -398,11 +401,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++o_waits[x];
                 tc_fence_after();
               }
-              if (!take(vslot)) { ok = false; break; }
               if (!mma_pv(x, vslot % C::kSlots, j == 0, ph)) { ok = false; break; }
               release(vslot);
               if (j + 1 < it.n(x)) {
-                if (!take(kslot)) { ok = false; break; }
                 mma_s(x, 0, kslot % C::kSlots);
                 release(kslot);
                 s_group_done();
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const uint32_t s_col = 128 * x, o_col = C::kTmO0 + x * D;
     const float sl2 = p.scale_log2;
-    uint32_t s_waits = 0, pv_waits = 0;
+    uint32_t s_waits = 0;  // S chunks of this warpgroup so far = its pv_done phases
     // After a failed wait the warpgroup keeps walking the items without
     // touching barriers or TMEM, so that both warpgroups still meet at the
     // named barriers of split items.
@@ -445,11 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.n(x) && ok; ++j) {
         bool okw = mbar_wait_w(&s_full[x], s_waits & 1, ctl, kErrWaitSoftmax);
         ++s_waits;
-        if (okw && j > 0) {
-          // O_X holds every chunk before j once P V(j-1) is done
-          okw = mbar_wait_w(&pv_done[x], pv_waits & 1, ctl, kErrWaitSoftmax);
-          ++pv_waits;
-        }
+        // O_X holds every chunk before j: one thread issues every MMA and
+        // commit, S(j) after P V(j-1), and a commit tracks the completion of
+        // all earlier MMAs of its thread, so s_full(j) implies pv_done(j-1),
+        // which is therefore not waited for
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
@@ -537,8 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue: O_X / l -> bf16 row, LSE
       bool oke = false;
       if (ok) {
-        oke = mbar_wait_w(&pv_done[x], pv_waits & 1, ctl, kErrWaitEpilogue);
-        ++pv_waits;
+        // the last chunk's phase: one pv_done phase per S chunk
+        oke = mbar_wait_w(&pv_done[x], (s_waits - 1) & 1, ctl, kErrWaitEpilogue);
         oke = __all_sync(0xffffffffu, oke);
       }
       if (it.split) {
