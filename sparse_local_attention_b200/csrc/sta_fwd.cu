@@ -429,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const uint32_t s_col = 128 * x, o_col = C::kTmO0 + x * D;
     const float sl2 = p.scale_log2;
-    uint32_t s_waits = 0;  // S chunks of this warpgroup so far = its pv_done phases
+    // S chunks of this warpgroup so far, and its pv_done phases (one per chunk)
+    uint32_t s_waits = 0, pv_waits = 0;
     // After a failed wait the warpgroup keeps walking the items without
     // touching barriers or TMEM, so that both warpgroups still meet at the
     // named barriers of split items.
@@ -448,8 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++s_waits;
         // O_X holds every chunk before j: one thread issues every MMA and
         // commit, S(j) after P V(j-1), and a commit tracks the completion of
-        // all earlier MMAs of its thread, so s_full(j) implies pv_done(j-1),
-        // which is therefore not waited for
+        // all earlier MMAs of its thread, so s_full(j) implies pv_done(j-1):
+        // that phase is counted, not waited for.  (The lone-block kernel
+        // derives the count from s_waits instead, which keeps it clear of
+        // spills at head dim 64.)
+        if (kMode == 0 && j > 0) ++pv_waits;
         okw = __all_sync(0xffffffffu, okw);
         if (!okw) { ok = false; break; }
         tc_fence_after();
@@ -537,8 +541,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue: O_X / l -> bf16 row, LSE
       bool oke = false;
       if (ok) {
-        // the last chunk's phase: one pv_done phase per S chunk
-        oke = mbar_wait_w(&pv_done[x], (s_waits - 1) & 1, ctl, kErrWaitEpilogue);
+        // the last chunk's phase
+        oke = mbar_wait_w(&pv_done[x], (kMode == 0 ? pv_waits : s_waits - 1) & 1, ctl, kErrWaitEpilogue);
+        ++pv_waits;
         oke = __all_sync(0xffffffffu, oke);
       }
       if (it.split) {
