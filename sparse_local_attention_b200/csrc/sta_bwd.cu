@@ -55,7 +55,7 @@ struct Roles {
   static_assert(kCols % 32 == 0, "whole 32-column TMEM loads");
 };
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kAugPanelBytes = 4096, kAugBlockBytes = 2 * kAugPanelBytes;  // see BwdParams::aug
+constexpr uint32_t kAugPanelBytes = 4096, kAugBlockBytes = kAugPanelBytes;  // see BwdParams::aug
 // pairs of exponentials (of every 8) that the dK/dV and the dQ elementwise
 // passes compute on the FMA pipe (exp2_fma2) instead of the MUFU
 constexpr int kEmuDkdv = 0, kEmuDq = 0;
@@ -127,18 +127,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     const long long bt = run / p.nqb;  // bh * n_tiles + tile
     const int o = (int)(run - bt * p.nqb) * kBM + (int)(r - run * kBM);
     const int bh = (int)(bt / g.n_tiles), tile = (int)(bt - (long long)bh * g.n_tiles);
-    // row i of the block's two operand panels: lanes 0 / 1 write the two
-    // halves of the LSE panel's row, lanes 2 / 3 those of the D panel's row
+    // row i of the block's operand panel: lanes 0 / 1 write its two halves
     const int i = (int)(r - run * kBM);
-    uint4 *cell = reinterpret_cast<uint4 *>(p.aug + run * kAugBlockBytes + (lane >> 1) * kAugPanelBytes +
-                                            (i / 8) * 256 + (lane & 1) * 128 + (i % 8) * 16);
+    uint4 *cell = reinterpret_cast<uint4 *>(p.aug + run * kAugBlockBytes + (i / 8) * 256 + (lane & 1) * 128 +
+                                            (i % 8) * 16);
     if (o >= g.tau) {
       // rows past the tile's end: P = dS = 0 (LSE = +inf, D = 0)
       if (lane == 0) {
         p.dd_t[r] = 0.f;
         p.lse2_t[r] = INFINITY;
       }
-      if (lane < 4) *cell = make_uint4(lane == 0 ? hi_lo_bf16(-1e30f) : 0u, 0u, 0u, 0u);
+      if (lane < 2) *cell = make_uint4(lane == 0 ? hi_lo_bf16(-1e30f) : 0u, 0u, 0u, 0u);
       continue;
     }
     const long long tok = token_row(g, p.tiled, bh, tile, o);
@@ -160,7 +159,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
       p.lse2_t[r] = lse * kLog2e;
     }
     // S^T + (-LSE / scale) times scale_log2 is S^T scale_log2 - LSE log2 e
-    if (lane < 4) *cell = make_uint4((lane & 1) ? 0u : hi_lo_bf16(lane == 0 ? -lse / p.scale : -acc), 0u, 0u, 0u);
+    if (lane < 2) *cell = lane == 0 ? make_uint4(hi_lo_bf16(-lse / p.scale), hi_lo_bf16(-acc), 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
@@ -178,12 +177,15 @@ struct DkvCfg {
   static constexpr uint32_t kPanel = kBM * 128;
   static constexpr bool kSep = D == 64;                    // P^T, dS^T in columns of their own
   using R = Roles<kSep ? 4 : 2>;                           // the in-place path assumes two warpgroups
-  static constexpr int kStages = D == 128 ? 2 : 4;
-  static constexpr uint32_t kStage = 2 * kTile + kAugBlockBytes;  // Q, dO, the block's LSE and D panels
-  static constexpr uint32_t kOnes = kAugPanelBytes;               // panel of rows (1, 1, 0, ..., 0)
+  static constexpr int kStages = D == 128 ? 2 : 5;
+  static constexpr uint32_t kStage = 2 * kTile + kAugBlockBytes;  // Q, dO, the block's LSE / D panel
+  // two selector panels: rows (1, 1, 0, ..., 0) pick -LSE / scale, rows
+  // (0, 0, 1, 1, 0, ..., 0) pick -D out of the block's panel
+  static constexpr uint32_t kOnes = 2 * kAugPanelBytes;
   // barriers: st_full[S] st_empty[S] kv_full kv_free s_full s_read p_ready pd_free acc_done acc_free drain
   static constexpr int kNumBars = 2 * kStages + 9;
   static constexpr uint32_t kSmem = 2 * kTile + kStages * kStage + kOnes + kNumBars * 8 + 64 + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmS = 0, kTmDP = 128;
   static constexpr uint32_t kTmP = kSep ? 256 : kTmS, kTmDS = kSep ? 320 : kTmDP;
   static constexpr uint32_t kTmDV = kSep ? 384 : 256, kTmDK = kTmDV + D;
@@ -238,11 +240,12 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // the panel of ones: row k = (1, 1, 0, ..., 0) in the first half, zeros in
-  // the second (layout of BwdParams::aug)
+  // the selector panels (layout of BwdParams::aug): every row of the first
+  // is (1, 1, 0, ..., 0), of the second (0, 0, 1, 1, 0, ..., 0)
   for (int c = threadIdx.x; c < (int)(C::kOnes / 16); c += blockDim.x) {
-    const bool first_half = ((c * 16) % 256) < 128;
-    reinterpret_cast<uint4 *>(ones_s)[c] = make_uint4(first_half ? 0x3F803F80u : 0u, 0u, 0u, 0u);
+    const bool first_half = ((c * 16) % 256) < 128, second_panel = c * 16 >= (int)kAugPanelBytes;
+    const uint32_t ones = first_half ? 0x3F803F80u : 0u;  // two bf16 1.0
+    reinterpret_cast<uint4 *>(ones_s)[c] = second_panel ? make_uint4(0u, ones, 0u, 0u) : make_uint4(ones, 0u, 0u, 0u);
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -311,8 +314,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
       const uint64_t kd = smem_desc_sw128(smem_u32(k_s), 16, 1024), vd = smem_desc_sw128(smem_u32(v_s), 16, 1024);
       const uint64_t sk0 = smem_desc_sw128(smem_u32(stages), 16, 1024);              // K-major Q / dO
       const uint64_t sm0 = smem_desc_sw128(smem_u32(stages), C::kPanel, 1024);       // MN-major Q / dO
-      const uint64_t ones_d = smem_desc_plain(smem_u32(ones_s), 128, 256);
-      const uint64_t aug0 = smem_desc_plain(smem_u32(stages + 2 * C::kTile), 128, 256);  // stage 0's LSE panel
+      const uint64_t ones_d = smem_desc_plain(smem_u32(ones_s), 128, 256);                    // selects -LSE / scale
+      const uint64_t ones_dd = smem_desc_plain(smem_u32(ones_s) + kAugPanelBytes, 128, 256);  // selects -D
+      const uint64_t aug0 = smem_desc_plain(smem_u32(stages + 2 * C::kTile), 128, 256);  // stage 0's LSE / D panel
       uint32_t ld = 0, item_ctr = 0, p_waits = 0, r_waits = 0;
       bool ok = true, issued = false;
       // S^T = K Q^T and dP^T = V dO^T for the chunk in stage `st`
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
           mma_ss_w(tmem + C::kTmDP, vd + off, sk0 + dso + off, idesc_ss, kk > 0 ? 1u : 0u);
         }
         // - D per query column
-        mma_ss_w(tmem + C::kTmDP, ones_d, aug0 + ((st * C::kStage + kAugPanelBytes) >> 4), idesc_ss, 1u);
+        mma_ss_w(tmem + C::kTmDP, ones_dd, aug0 + ((st * C::kStage) >> 4), idesc_ss, 1u);
         mma_commit_w(s_full);
       };
       auto wait_stage = [&](uint32_t l) -> bool {

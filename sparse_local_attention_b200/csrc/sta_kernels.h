@@ -73,12 +73,13 @@ struct BwdParams {
   const void *o, *dout;  // preprocess inputs
   const float *lse;      // forward LSE (natural log)
   float *lse2_t, *dd_t;  // one 128-float run per query block: LSE*log2(e), D = rowsum(dO*O)
-  // Per query block, two 4 KB K-major operand panels (no swizzle; 16 groups
+  // Per query block, one 4 KB K-major operand panel (no swizzle; 16 groups
   // of 8 rows at 256 bytes, the two 8-element halves of a row 128 bytes
-  // apart): row q holds (hi, lo, 0, ..., 0) with hi + lo = -LSE_q*log2(e) /
-  // scale_log2 (first panel) and -D_q (second), hi and lo bf16.  The dK/dV
-  // kernel adds them to S^T and dP^T with one more K step against a panel of
-  // ones, so that its elementwise pass needs no per-query operand.
+  // apart): row q holds (a_hi, a_lo, d_hi, d_lo, 0, ..., 0) with a_hi + a_lo
+  // = -LSE_q*log2(e) / scale_log2 and d_hi + d_lo = -D_q, all bf16.  The
+  // dK/dV kernel adds them to S^T and dP^T with one more K step each, against
+  // panels whose rows are (1, 1, 0, ...) and (0, 0, 1, 1, 0, ...), so that its
+  // elementwise pass needs no per-query operand.
   uint8_t *aug;
   void *dq, *dk, *dv;    // bf16 outputs
   const int32_t *kv_list, *kv_count;  // forward lists (dQ kernel)
