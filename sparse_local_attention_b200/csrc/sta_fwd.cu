@@ -27,7 +27,11 @@
 //     runs the softmax of chunk j, the tensor core computes S_B(j), and so on.
 //     P_X is written over the first 64 columns of S_X; tcgen05.mma operations
 //     issued by one thread execute in order, so P V(j) has read P before the
-//     S of chunk j + 1 overwrites that buffer.
+//     S of chunk j + 1 overwrites that buffer.  What stands between the end
+//     of a block's softmax pass and its next S is kept short: the ring slots
+//     of a chunk are waited for before the softmax finishes, the P V products
+//     of the first kLeadKeys keys are issued as soon as their P is written,
+//     and the softmax takes S(j)'s arrival as proof that P V(j-1) is done.
 //   * warps 0-3 / 4-7: softmax of block A / B.  Query row r lives in TMEM lane
 //     r and a thread owns one whole row: row max and sum need no shuffles.
 //     fp32 online softmax in the log2 domain with lazy rescaling of O (only
