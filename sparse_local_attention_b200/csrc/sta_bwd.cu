@@ -549,6 +549,7 @@ struct DqCfg {
   // barriers: full[S] empty[S] q_full q_free s_full s_read ds_ready ds_free acc_done acc_free drain
   static constexpr int kNumBars = 2 * kSlots + 9;
   static constexpr uint32_t kSmem = (2 + kSlots) * kTile + kNumBars * 8 + 64 + 16 + kMaxCoords * 16 + 1024;
+  static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
   static constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDS = 256, kTmDQ = 320;
   static_assert(kTmDQ + D <= 512, "TMEM budget");
 };
