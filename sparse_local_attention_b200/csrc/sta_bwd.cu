@@ -9,7 +9,9 @@
 //
 // Three launches, no atomics (the result is deterministic):
 //   1. bwd_pre: D and LSE * log2(e) per query row, stored tile-major so a
-//      128-row block reads them as one contiguous run.
+//      128-row block reads them as one contiguous run, and per query block
+//      the operand panel that carries -LSE / scale and -D into the dK/dV
+//      kernel's products (BwdParams::aug).
 //   2. bwd_dkdv: one 128-row key block per work item (key-block major).  K and
 //      V stay in shared memory; the query blocks of every query tile whose
 //      window holds the key tile (the planner's inverse lists) stream through
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::R::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *k_s = smem, *v_s = smem + C::kTile;
-  uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, LSE panel, D panel}
+  uint8_t *stages = smem + 2 * C::kTile;  // [stage]{Q tile, dO tile, LSE / D panel}
   uint8_t *ones_s = stages + C::kStages * C::kStage;
   uint64_t *bars = reinterpret_cast<uint64_t *>(ones_s + C::kOnes);
   uint64_t *st_full = bars, *st_empty = bars + C::kStages;
