@@ -147,7 +147,8 @@ sta_status sta_plan_geometry(sta_plan_t plan, int32_t *n_tiles, int32_t *tile_vo
  *       built without STA_PROBLEM_BACKWARD.
  * *n_items receives the item count (out may be NULL to query it; otherwise
  * cap_items must be >= *n_items, else STA_ERR_INVALID_ARG).  n_lone may be
- * NULL.  This call has no counterpart in the paper. */
+ * NULL.  This call has no counterpart in the method's description
+ * ("Fast Video Generation with Sliding Tile Attention"). */
 #define STA_WORK_FORWARD 0
 #define STA_WORK_FORWARD_HOST 1
 #define STA_WORK_DKDV 2
@@ -160,7 +161,8 @@ sta_status sta_plan_work_items(sta_plan_t plan, int32_t which, int32_t *out, siz
  * `backward` is 0 for a plan built without STA_PROBLEM_BACKWARD).  For sizing
  * CUDA-graph captures and for launch accounting.  Either pointer may be NULL;
  * host-only plans report what a device plan of the same problem launches.
- * This call has no counterpart in the paper. */
+ * This call has no counterpart in the method's description
+ * ("Fast Video Generation with Sliding Tile Attention"). */
 sta_status sta_plan_launches(sta_plan_t plan, int32_t *forward, int32_t *backward);
 
 /* Token permutation between raster and tile-major order for a bf16 tensor
@@ -183,7 +185,8 @@ sta_status sta_forward(sta_plan_t plan, const void *q, const void *k, const void
 
 /* Device workspace that sta_forward_host needs: device copies of q, k, v, o
  * and lse, then sta_forward's own workspace.  This call has no counterpart in
- * the paper. */
+ * the method's description ("Fast Video Generation with Sliding Tile
+ * Attention"). */
 sta_status sta_plan_host_workspace_size(sta_plan_t plan, size_t *bytes);
 
 /* Forward pass on HOST tensors (same computation and layouts as sta_forward):
@@ -198,7 +201,9 @@ sta_status sta_plan_host_workspace_size(sta_plan_t plan, size_t *bytes);
  * the call, o and lse are in host memory.  Copies overlap only for page-locked
  * host memory.  With tiles that are not TMA boxes of the raster tensor, the
  * whole tensors are copied in, computed and copied out in order.  Host buffers must stay valid and unchanged until
- * `stream` has passed the call.  This call has no counterpart in the paper. */
+ * `stream` has passed the call.  This call has no counterpart in the
+ * method's description ("Fast Video Generation with Sliding Tile
+ * Attention"). */
 sta_status sta_forward_host(sta_plan_t plan, const void *q, const void *k, const void *v, void *o, float *lse,
                             void *workspace, size_t workspace_bytes, void *stream, uint32_t flags);
 
@@ -216,8 +221,9 @@ sta_status sta_backward(sta_plan_t plan, const void *q, const void *k, const voi
                         void *dv, void *workspace, size_t workspace_bytes, void *stream,
                         uint32_t flags);
 
-/* sta_backward without a caller workspace.  (No counterpart in the paper: this
- * is a calling convention of this library.)  Meant for callers that cannot
+/* sta_backward without a caller workspace.  (No counterpart in the method's
+ * description: this is a calling convention of this library.)  Meant for
+ * callers that cannot
  * allocate device memory where they run the backward pass -- for example when
  * a framework's caching allocator already owns the whole device, or on a path
  * where the memory footprint must not change once set up -- and so cannot hand
