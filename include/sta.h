@@ -224,8 +224,8 @@ sta_status sta_backward(sta_plan_t plan, const void *q, const void *k, const voi
 /* sta_backward without a caller workspace.  (No counterpart in the method's
  * description: this is a calling convention of this library.)  Meant for
  * callers that cannot allocate device memory where they run the backward
- * pass -- for example when
- * a framework's caching allocator already owns the whole device, or on a path
+ * pass -- for example when a framework's caching allocator already owns the
+ * whole device, or on a path
  * where the memory footprint must not change once set up -- and so cannot hand
  * over a workspace.  The temporaries go to a file-scope device array of 32 MiB
  * inside libsta.so instead; every GPU that loads the library holds that array
