@@ -193,7 +193,7 @@ sta_status sta_plan_host_workspace_size(sta_plan_t plan, size_t *bytes);
  * q, k, v are read from host memory and o (and lse, nullable) written to host
  * memory; `workspace` is device memory of at least
  * sta_plan_host_workspace_size bytes, 16-byte aligned.  The (batch, head)
- * slices are processed in up to 8 groups: the inputs of one group are copied
+ * slices are processed in up to 24 groups: the inputs of one group are copied
  * to the device while the previous group is computed, and each group's
  * outputs are copied back while later groups run, on two internal streams
  * ordered against `stream` with events (one cudaMemcpyAsync per tensor and

@@ -90,7 +90,7 @@ size_t bwd_vec_bytes(const sta_plan_s *pl) { return bwd_blocks(pl) * 128 * 4; }
 constexpr size_t kAugBytesPerBlock = 4096;
 // sta_forward_host workspace: device copies of Q, K, V, O and LSE (each at a
 // 256-byte boundary), then sta_forward's own workspace (status word first).
-constexpr int kHostGroups = 8;  // slice groups pipelined by sta_forward_host
+constexpr int kHostGroups = 24;  // slice groups pipelined by sta_forward_host
 
 
 size_t lse_bytes(const sta_plan_s *pl) { return (size_t)pl->g.B * pl->g.Hh * pl->g.N * 4; }

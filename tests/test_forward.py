@@ -231,7 +231,7 @@ def _host_vs_device(plan, q, k, v, pinned):
 
 
 def test_forward_host_full_scale_groups():
-    """32 slices in 8 groups of 4 (fine-tuning shapes): the pipelined host call
+    """32 slices in 24 groups of one or two (fine-tuning shapes): the pipelined host call
     returns exactly the device call's outputs."""
     wl = WORKLOADS["finetune"]
     q, k, v = make_inputs(wl, seed=6)

@@ -85,7 +85,7 @@ def test_host_items_are_the_forward_items_by_slice_group(name):
     host, _ = sta.sta_plan_work_items(plan, sta.STA_WORK_FORWARD_HOST)
     assert sorted(map(tuple, items.tolist())) == sorted(map(tuple, host.tolist()))
     slices = wl.B * wl.Hh
-    groups = min(slices, 8)
+    groups = min(slices, 24)
     group_of = {}
     for g in range(groups):
         for s in range(slices * g // groups, slices * (g + 1) // groups):
