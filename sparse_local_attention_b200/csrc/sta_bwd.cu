@@ -118,50 +118,52 @@ __device__ __forceinline__ void quarters_pipelined(uint32_t s_addr, uint32_t dp_
 }
 
 // ----------------------------------------------------------------------- 1. preprocess
+// A group of D / 8 lanes per row (16-byte loads of O and dO, the row's LSE
+// loaded beside them), 32 / (D / 8) rows per warp and iteration.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   const Geometry &g = p.g;
-  const int lane = threadIdx.x & 31;
-  const long long nrows = (long long)g.B * g.Hh * g.n_tiles * p.nqb * kBM;  // padded runs
-  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
-  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < nrows; r += warps) {
+  constexpr int kLanes = D / 8, kRows = 32 / kLanes;
+  static_assert(kLanes >= 2 && kLanes <= 32 && 32 % kLanes == 0, "whole rows per warp");
+  const int lane = threadIdx.x & 31, sub = lane / kLanes, part = lane % kLanes;
+  const long long nrows = (long long)g.B * g.Hh * g.n_tiles * p.nqb * kBM;  // padded runs, a multiple of kRows
+  const long long step = (long long)gridDim.x * (blockDim.x / 32) * kRows;
+  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32 * kRows + sub; r < nrows; r += step) {
     const long long run = r / kBM;
     const long long bt = run / p.nqb;  // bh * n_tiles + tile
     const int o = (int)(run - bt * p.nqb) * kBM + (int)(r - run * kBM);
     const int bh = (int)(bt / g.n_tiles), tile = (int)(bt - (long long)bh * g.n_tiles);
-    // row i of the block's operand panel: lanes 0 / 1 write its two halves
-    const int i = (int)(r - run * kBM);
-    uint4 *cell = reinterpret_cast<uint4 *>(p.aug + run * kAugBlockBytes + (i / 8) * 256 + (lane & 1) * 128 +
-                                            (i % 8) * 16);
-    if (o >= g.tau) {
-      // rows past the tile's end: P = dS = 0 (LSE = +inf, D = 0)
-      if (lane == 0) {
-        p.dd_t[r] = 0.f;
-        p.lse2_t[r] = INFINITY;
+    // rows past the tile's end: P = dS = 0 (LSE = +inf, D = 0)
+    const bool valid = o < g.tau;
+    float acc = 0.f, lse = 0.f;
+    if (valid) {
+      const long long tok = token_row(g, p.tiled, bh, tile, o);
+      const uint4 a = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.o) + tok * D)[part];
+      const uint4 b = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.dout) + tok * D)[part];
+      if (part == 0) lse = p.lse[tok];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&av[e]));
+        const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&bv[e]));
+        acc = fmaf(af.x, bf.x, fmaf(af.y, bf.y, acc));
       }
-      if (lane < 2) *cell = make_uint4(lane == 0 ? hi_lo_bf16(-1e30f) : 0u, 0u, 0u, 0u);
-      continue;
     }
-    const long long tok = token_row(g, p.tiled, bh, tile, o);
-    const __nv_bfloat16 *orow = static_cast<const __nv_bfloat16 *>(p.o) + tok * D;
-    const __nv_bfloat16 *drow = static_cast<const __nv_bfloat16 *>(p.dout) + tok * D;
-    float acc = 0.f;
+    // sum over the row's lane group (every lane of the warp takes part)
 #pragma unroll
-    for (int e = 0; e < D / 64; ++e) {
-      const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162 *>(orow)[lane + 32 * e];
-      const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162 *>(drow)[lane + 32 * e];
-      const float2 af = __bfloat1622float2(a), bf = __bfloat1622float2(b);
-      acc = fmaf(af.x, bf.x, fmaf(af.y, bf.y, acc));
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (part == 0) {
+      p.dd_t[r] = valid ? acc : 0.f;
+      p.lse2_t[r] = valid ? lse * kLog2e : INFINITY;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    const float lse = p.lse[tok];
-    if (lane == 0) {
-      p.dd_t[r] = acc;
-      p.lse2_t[r] = lse * kLog2e;
-    }
+    // row i of the block's operand panel: parts 0 / 1 write its two halves;
     // S^T + (-LSE / scale) times scale_log2 is S^T scale_log2 - LSE log2 e
-    if (lane < 2) *cell = lane == 0 ? make_uint4(hi_lo_bf16(-lse / p.scale), hi_lo_bf16(-acc), 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    if (part < 2) {
+      const int i = (int)(r - run * kBM);
+      uint4 *cell = reinterpret_cast<uint4 *>(p.aug + run * kAugBlockBytes + (i / 8) * 256 + part * 128 + (i % 8) * 16);
+      *cell = part == 0 ? make_uint4(hi_lo_bf16(valid ? -lse / p.scale : -1e30f), valid ? hi_lo_bf16(-acc) : 0u, 0u, 0u)
+                        : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 }
 
@@ -884,7 +886,8 @@ cudaError_t launch_bwd_d(const BwdParams &p, const CUtensorMap &tq, const CUtens
     attr_set = true;
   }
   const long long rows = (long long)p.g.B * p.g.Hh * p.g.N;
-  long long pre_blocks = (rows + 7) / 8;
+  constexpr int kPreRows = 8 * (32 / (D / 8));  // rows per 256-thread block and iteration
+  long long pre_blocks = (rows + kPreRows - 1) / kPreRows;
   if (pre_blocks > (long long)num_sms * 16) pre_blocks = (long long)num_sms * 16;
   bwd_pre_kernel<D><<<(int)pre_blocks, 256, 0, stream>>>(p);
   const int g1 = p.n_work_kv < num_sms ? p.n_work_kv : num_sms;
